@@ -1,0 +1,361 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix,
+never against a retyped copy of the oracle's own formula.  CPU only."""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from lens_inputs import LENS, TINY, f32_to_bf16_bits, make_weights, weight_specs
+from oracle import lens_oracle as o
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    rows = [l.split() for l in open(os.path.join(GOLDEN, name)) if l.strip() and not l.startswith("#")]
+    return rows
+
+
+@pytest.fixture(scope="module")
+def tinyW():
+    return o.Weights(make_weights(TINY, seed=11, std=0.2, bias_std=0.05, gain_std=0.2))
+
+
+# ------------------------------------------------------------------ model size
+def test_param_count_matches_blog_arithmetic():
+    g = {k: float(v) for k, v in _golden("lens_param_arithmetic.txt")}
+    pc = o.param_count(LENS)
+    D, F = LENS.hidden, LENS.mlp_hidden
+    assert abs(4 * D * D / 1e6 - g["attn_proj_M"]) < 0.01
+    assert abs(3 * D * F / 1e6 - g["mlp_M"]) < 0.1
+    # the page adds rounded parts (28.2 + 14.1), so allow its rounding
+    assert abs(pc["stream_weights"] / 1e6 - g["stream_M"]) / g["stream_M"] < 0.005
+    assert abs(2 * pc["stream_weights"] / 1e6 - g["block_M"]) / g["block_M"] < 0.005
+    assert abs(pc["total"] * 2 / 1e9 - g["bf16_GB"]) < 0.05
+    # the synthetic tensor list holds exactly these parameters
+    assert sum(int(np.prod(s)) for _, s, _ in weight_specs(LENS)) == pc["total"]
+
+
+# ------------------------------------------------------------------ patchify
+def test_patchify_roundtrip_and_grouping():
+    rng = np.random.default_rng(0)
+    Z = rng.standard_normal((2, 32, 6, 10)).astype(np.float32)
+    X = o.patchify(Z)
+    assert X.shape == (2, 15, 128)                       # 2*2*32 = 128 per token
+    assert np.array_equal(o.unpatchify(X, 3, 5, 32), Z)  # bijection, bit-exact
+    # token (i, j) holds exactly the 2x2 spatial block at (2i.., 2j..) of every channel
+    for b in range(2):
+        for i in range(3):
+            for j in range(5):
+                blk = Z[b, :, 2 * i:2 * i + 2, 2 * j:2 * j + 2].ravel()
+                assert sorted(X[b, i * 5 + j].tolist()) == sorted(blk.tolist())
+    # reading: features channel-major, then patch row, then patch column
+    assert X[1, 7, 4 * 3 + 2 * 1 + 0] == Z[1, 3, 2 * 1 + 1, 2 * 2 + 0]
+
+
+# ------------------------------------------------------------------ RoPE
+def test_rope_axes_cover_head_dim():
+    assert sum(LENS.rope_axes) == LENS.head_dim == 64
+
+
+def test_rope_complex_brute_force():
+    """Rotation of pair k equals multiplying (x0 + i x1) by exp(i angle)."""
+    rng = np.random.default_rng(1)
+    ids = rng.integers(0, 50, size=(7, 3))
+    ang = o.rope_angles(ids, (8, 28, 28), 1e4)
+    x = rng.standard_normal((7, 64))
+    y = o.apply_rope(x, ang)
+    for n in range(7):
+        for k in range(32):
+            c = complex(x[n, 2 * k], x[n, 2 * k + 1]) * complex(math.cos(ang[n, k]), math.sin(ang[n, k]))
+            assert abs(y[n, 2 * k] - c.real) < 1e-12 and abs(y[n, 2 * k + 1] - c.imag) < 1e-12
+    # the first pair of each axis turns by exactly pos (omega = 1); the axis owns its segment
+    assert np.allclose(ang[:, 0], ids[:, 0]) and np.allclose(ang[:, 4], ids[:, 1]) and np.allclose(ang[:, 18], ids[:, 2])
+
+
+def test_rope_norm_identity_and_relative_position():
+    rng = np.random.default_rng(2)
+    ids = o.position_ids(5, 7, 3)
+    ang = o.rope_angles(ids, (8, 28, 28), 1e4)
+    q = rng.standard_normal((ids.shape[0], 64))
+    k = rng.standard_normal((ids.shape[0], 64))
+    rq, rk = o.apply_rope(q, ang), o.apply_rope(k, ang)
+    assert np.allclose(np.linalg.norm(rq, axis=1), np.linalg.norm(q, axis=1), rtol=0, atol=1e-12)
+    assert np.array_equal(rq[:3], q[:3])       # text ids (0,0,0): identity
+    # <R(p) q, R(p') k> depends only on p - p': shift every id by a constant
+    ang2 = o.rope_angles(ids + np.array([3, 11, 5]), (8, 28, 28), 1e4)
+    d1 = o.apply_rope(q, ang) @ o.apply_rope(k, ang).T
+    d2 = o.apply_rope(q, ang2) @ o.apply_rope(k, ang2).T
+    assert np.allclose(d1, d2, rtol=0, atol=1e-9)
+    # a displacement along the width axis moves only dims [36, 64)
+    a0 = o.rope_angles(np.array([[0, 2, 3]]), (8, 28, 28), 1e4)
+    a1 = o.rope_angles(np.array([[0, 2, 4]]), (8, 28, 28), 1e4)
+    x = rng.standard_normal((1, 64))
+    diff = np.abs(o.apply_rope(x, a0) - o.apply_rope(x, a1))[0]
+    assert diff[:36].max() == 0 and diff[36:].max() > 0
+
+
+def test_position_ids_layout():
+    ids = o.position_ids(2, 3, 2)
+    assert ids.tolist() == [[0, 0, 0], [0, 0, 0], [0, 0, 0], [0, 0, 1], [0, 0, 2], [0, 1, 0], [0, 1, 1], [0, 1, 2]]
+
+
+# ------------------------------------------------------------------ norms, activations, sinusoid
+def test_rms_norm_and_silu_closed_forms():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((4, 33)) * 7.0
+    y = o.rms_norm(x, 0.0)
+    assert np.allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, atol=1e-12)
+    assert np.allclose(o.rms_norm(5.0 * x, 0.0), y, atol=1e-12)
+    g = rng.standard_normal(33)
+    assert np.allclose(o.rms_norm(x, 0.0, g), y * g, atol=1e-12)
+    assert o.silu(np.array(0.0)) == 0.0
+    assert abs(o.silu(np.array(1.0)) - 0.7310585786300049) < 1e-15      # 1 / (1 + e^-1)
+    assert abs(o.silu(np.array(40.0)) - 40.0) < 1e-12
+    assert abs(o.silu(np.array(-40.0))) < 1e-15
+
+
+def test_timestep_features():
+    e0 = o.timestep_features(np.array([0.0]), 256)[0]
+    assert np.array_equal(e0, np.r_[np.ones(128), np.zeros(128)])
+    t = 0.37
+    e = o.timestep_features(np.array([t]), 256)[0]
+    assert abs(e[0] - math.cos(370.0)) < 1e-12 and abs(e[128] - math.sin(370.0)) < 1e-12
+    # lowest frequency is 10000^(-127/128)
+    assert abs(e[127] - math.cos(370.0 * 10000 ** (-127 / 128))) < 1e-12
+    assert np.allclose(e[:128] ** 2 + e[128:] ** 2, 1.0)
+
+
+# ------------------------------------------------------------------ attention
+def _attn_loops(q, k, v):
+    Nq, d = q.shape
+    out = np.zeros((Nq, v.shape[1]))
+    for i in range(Nq):
+        s = [sum(q[i, c] * k[j, c] for c in range(d)) / math.sqrt(d) for j in range(k.shape[0])]
+        m = max(s)
+        w = [math.exp(x - m) for x in s]
+        z = sum(w)
+        for j in range(k.shape[0]):
+            out[i] += w[j] / z * v[j]
+    return out
+
+
+def test_attention_brute_force_and_invariances():
+    rng = np.random.default_rng(4)
+    q, k, v = (rng.standard_normal((1, 2, 5, 4)) * 2 for _ in range(3))
+    out = o.attention(q, k, v)
+    for h in range(2):
+        assert np.allclose(out[0, h], _attn_loops(q[0, h], k[0, h], v[0, h]), atol=1e-12)
+    perm = rng.permutation(5)
+    assert np.allclose(o.attention(q, k[:, :, perm], v[:, :, perm]), out, atol=1e-12)
+    assert np.allclose(o.attention(q[:, :, perm], k, v), out[:, :, perm], atol=1e-12)
+    assert np.allclose(o.attention(np.zeros_like(q), k, v), v.mean(axis=2, keepdims=True), atol=1e-12)
+
+
+# ------------------------------------------------------------------ text input
+def test_text_input_per_layer_normalisation(tinyW):
+    rng = np.random.default_rng(5)
+    E = rng.standard_normal((2, 3, 4, TINY.txt_dim))
+    c = o.text_input(tinyW, E, 0.0)
+    E2 = E.copy()
+    E2[:, :, 2, :] *= 9.0                       # each layer slice is normalised on its own
+    assert np.allclose(o.text_input(tinyW, E2, 0.0), c, atol=1e-9)
+    E3 = E.copy()
+    E3[:, :, :, :] *= np.array([1, 2, 3, 4])[None, None, :, None]   # unequal per-layer scales:
+    assert np.allclose(o.text_input(tinyW, E3, 0.0), c, atol=1e-9)
+    z = o.text_input(tinyW, np.zeros_like(E), TINY.eps)
+    assert np.allclose(z, tinyW("txt_in.bias")[None, None, :], atol=1e-15)
+
+
+# ------------------------------------------------------------------ block
+def _block_inputs(dims, B=2, Ni=6, Nt=3, seed=6):
+    rng = np.random.default_rng(seed)
+    h_img = rng.standard_normal((B, Ni, dims.hidden))
+    h_txt = rng.standard_normal((B, Nt, dims.hidden)) * 2
+    temb = rng.standard_normal((B, dims.hidden))
+    return h_img, h_txt, temb
+
+
+def _edit(W, fn):
+    t = dict(W.t)
+    fn(t)
+    return o.Weights(t)
+
+
+def _zero_rows(t, name, lo, hi):
+    w = t[name + ".weight"].copy(); w[lo:hi] = 0; t[name + ".weight"] = w
+    b = t[name + ".bias"].copy(); b[lo:hi] = 0; t[name + ".bias"] = b
+
+
+def test_block_zero_gates_is_identity(tinyW):
+    D = TINY.hidden
+
+    def zero_gates(t):
+        for s in ("img_mod", "txt_mod"):
+            _zero_rows(t, f"transformer_blocks.0.{s}", 2 * D, 3 * D)
+            _zero_rows(t, f"transformer_blocks.0.{s}", 5 * D, 6 * D)
+    W = _edit(tinyW, zero_gates)
+    h_img, h_txt, temb = _block_inputs(TINY)
+    ang = o.rope_angles(o.position_ids(2, 3, 3), TINY.rope_axes, TINY.rope_theta)
+    hi, ht = o.block(W, 0, h_img, h_txt, temb, ang, TINY.heads, TINY.eps)
+    assert np.array_equal(hi, h_img) and np.array_equal(ht, h_txt)
+
+
+def test_block_gate_linearity(tinyW):
+    """With the MLP gate closed the update is linear in the attention gate."""
+    D = TINY.hidden
+
+    def setup(scale):
+        def fn(t):
+            for s in ("img_mod", "txt_mod"):
+                _zero_rows(t, f"transformer_blocks.0.{s}", 5 * D, 6 * D)
+                w = o.upcast(t[f"transformer_blocks.0.{s}.weight"], np.float32)
+                b = o.upcast(t[f"transformer_blocks.0.{s}.bias"], np.float32)
+                w[2 * D:3 * D] *= scale; b[2 * D:3 * D] *= scale   # exact in bf16 (power of 2)
+                t[f"transformer_blocks.0.{s}.weight"] = f32_to_bf16_bits(w)
+                t[f"transformer_blocks.0.{s}.bias"] = f32_to_bf16_bits(b)
+        return _edit(tinyW, fn)
+    h_img, h_txt, temb = _block_inputs(TINY)
+    ang = o.rope_angles(o.position_ids(2, 3, 3), TINY.rope_axes, TINY.rope_theta)
+    a1 = o.block(setup(1.0), 0, h_img, h_txt, temb, ang, TINY.heads, TINY.eps)
+    a2 = o.block(setup(2.0), 0, h_img, h_txt, temb, ang, TINY.heads, TINY.eps)
+    assert np.allclose(a2[0] - h_img, 2 * (a1[0] - h_img), atol=1e-12)
+    assert np.allclose(a2[1] - h_txt, 2 * (a1[1] - h_txt), atol=1e-12)
+    assert np.abs(a1[0] - h_img).max() > 1e-3
+
+
+def test_block_stream_symmetry(tinyW):
+    """With identical weights in both streams the joint block treats [text; image]
+    symmetrically: swapping the streams (and their positions) swaps the outputs."""
+    def tie(t):
+        p = "transformer_blocks.0."
+        for a, b in (("img_mod", "txt_mod"), ("attn.img_qkv", "attn.txt_qkv"), ("attn.to_out", "attn.to_add_out"),
+                     ("img_mlp.w1", "txt_mlp.w1"), ("img_mlp.w2", "txt_mlp.w2"), ("img_mlp.w3", "txt_mlp.w3")):
+            t[p + b + ".weight"] = t[p + a + ".weight"]; t[p + b + ".bias"] = t[p + a + ".bias"]
+        t[p + "attn.norm_added_q.weight"] = t[p + "attn.norm_q.weight"]
+        t[p + "attn.norm_added_k.weight"] = t[p + "attn.norm_k.weight"]
+    W = _edit(tinyW, tie)
+    h_img, h_txt, temb = _block_inputs(TINY, Ni=4, Nt=4)
+    rng = np.random.default_rng(7)
+    ang = rng.uniform(-3, 3, size=(8, TINY.head_dim // 2))
+    hi, ht = o.block(W, 0, h_img, h_txt, temb, ang, TINY.heads, TINY.eps)
+    ang_sw = np.concatenate([ang[4:], ang[:4]])
+    hi2, ht2 = o.block(W, 0, h_txt, h_img, temb, ang_sw, TINY.heads, TINY.eps)
+    assert np.allclose(hi2, ht, atol=1e-10) and np.allclose(ht2, hi, atol=1e-10)
+
+
+def test_block_token_permutation_equivariance(tinyW):
+    h_img, h_txt, temb = _block_inputs(TINY, Ni=6, Nt=3)
+    ang = o.rope_angles(o.position_ids(2, 3, 3), TINY.rope_axes, TINY.rope_theta)
+    hi, ht = o.block(tinyW, 0, h_img, h_txt, temb, ang, TINY.heads, TINY.eps)
+    perm = np.array([4, 0, 5, 2, 1, 3])
+    ang_p = np.concatenate([ang[:3], ang[3:][perm]])
+    hi_p, ht_p = o.block(tinyW, 0, h_img[:, perm], h_txt, temb, ang_p, TINY.heads, TINY.eps)
+    assert np.allclose(hi_p, hi[:, perm], atol=1e-10) and np.allclose(ht_p, ht, atol=1e-10)
+
+
+def test_block_single_token_attention_is_value(tinyW):
+    """One token in total: softmax weight 1, so the attention output is that token's v
+    (after nothing: RoPE never touches v)."""
+    D, H = TINY.hidden, TINY.heads
+    rng = np.random.default_rng(8)
+    h_txt = rng.standard_normal((1, 1, D))
+    h_img = np.zeros((1, 0, D))
+    temb = rng.standard_normal((1, D))
+    ang = rng.uniform(-3, 3, size=(1, TINY.head_dim // 2))
+
+    def no_mlp(t):
+        _zero_rows(t, "transformer_blocks.0.txt_mod", 5 * D, 6 * D)
+    W = _edit(tinyW, no_mlp)
+    _, ht = o.block(W, 0, h_img, h_txt, temb, ang, H, TINY.eps)
+    m = o.linear(W, "transformer_blocks.0.txt_mod", o.silu(temb))
+    sh, sc, g = m[:, :D], m[:, D:2 * D], m[:, 2 * D:3 * D]
+    a = (1 + sc) * h_txt[0] / np.sqrt(np.mean(h_txt[0] ** 2) + TINY.eps) + sh
+    v = o.linear(W, "transformer_blocks.0.attn.txt_qkv", a)[:, 2 * D:]
+    ref = h_txt[0] + g * o.linear(W, "transformer_blocks.0.attn.to_add_out", v)
+    assert np.allclose(ht[0], ref, atol=1e-10)
+
+
+def test_block_row_selection_matches_full(tinyW):
+    h_img, h_txt, temb = _block_inputs(TINY, Ni=6, Nt=3)
+    ang = o.rope_angles(o.position_ids(2, 3, 3), TINY.rope_axes, TINY.rope_theta)
+    hi, ht = o.block(tinyW, 0, h_img, h_txt, temb, ang, TINY.heads, TINY.eps)
+    hs, ts = o.block(tinyW, 0, h_img, h_txt, temb, ang, TINY.heads, TINY.eps,
+                     img_rows=np.array([5, 1]), txt_rows=np.array([2]))
+    assert np.allclose(hs, hi[:, [5, 1]], atol=1e-12) and np.allclose(ts, ht[:, [2]], atol=1e-12)
+
+
+def test_forward_runs_tiny(tinyW):
+    rng = np.random.default_rng(9)
+    X = rng.standard_normal((2, 6, TINY.in_channels))
+    E = f32_to_bf16_bits(rng.standard_normal((2, 3, 4, TINY.txt_dim)).astype(np.float32))
+    v = o.forward(tinyW, TINY, X, 2, 3, E, [0.3, 0.9])
+    assert v.shape == (2, 6, TINY.in_channels) and np.all(np.isfinite(v))
+    # batch elements are independent
+    v1 = o.forward(tinyW, TINY, X[1:], 2, 3, E[1:], [0.9])
+    assert np.allclose(v1[0], v[1], atol=1e-12)
+
+
+# ------------------------------------------------------------------ sampler
+def test_euler_lands_on_data_for_straight_paths():
+    """x_t = (1-t) x0 + t x1 with v = x1 - x0: Euler is exact on straight lines."""
+    rng = np.random.default_rng(10)
+    x0, x1 = rng.standard_normal((2, 3, 8))
+    vel = lambda x, t, c: x1 - x0
+    for S in (1, 2, 4, 7, 20):
+        assert np.allclose(o.sample_euler(vel, x1, S, 1.0), x0, atol=1e-12)
+    # one step from t = 1 lands exactly on x0
+    assert np.allclose(o.euler(x1, x1 - x0, 1.0), x0, atol=1e-15)
+    # the exact velocity of the straight path at (x_t, t) is (x_t - x0) / t
+    vel2 = lambda x, t, c: (x - x0) / t
+    assert np.allclose(o.sample_euler(vel2, x1, 5, 1.0), x0, atol=1e-12)
+    assert o.timesteps(4).tolist() == [1.0, 0.75, 0.5, 0.25]
+
+
+def test_cfg_special_scales():
+    rng = np.random.default_rng(11)
+    c, u = rng.standard_normal((2, 10))
+    assert np.allclose(o.cfg_combine(c, u, 1.0), c, atol=1e-15)
+    assert np.array_equal(o.cfg_combine(c, u, 0.0), u)
+    assert np.allclose(o.cfg_combine(c, u, 5.0), u + 5 * (c - u))
+    calls = []
+    vel = lambda x, t, cond: (calls.append(cond), np.full_like(x, 1.0 if cond else 3.0))[1]
+    x = o.sample_euler(vel, np.zeros(4), 2, 5.0)          # v = 3 + 5 (1 - 3) = -7 each step
+    assert np.allclose(x, 7.0) and calls.count(False) == 2
+    calls.clear()
+    o.sample_euler(vel, np.zeros(4), 2, 1.0)
+    assert calls.count(False) == 0                        # guidance 1: no unconditional pass
+
+
+# ------------------------------------------------------------------ noise
+def test_splitmix64_published_vectors():
+    want = [int(r[0], 16) for r in _golden("splitmix64_seed0.txt")]
+    gamma = 0x9E3779B97F4A7C15
+    states = np.array([0, gamma, (2 * gamma) % 2 ** 64], np.uint64)
+    assert [int(x) for x in o.splitmix64(states)] == want
+
+
+def test_noise_is_standard_normal():
+    from scipy import stats
+    z = o.noise(42, 200_000).astype(np.float64)
+    assert np.all(np.isfinite(z))
+    assert abs(z.mean()) < 0.01 and abs(z.var() - 1) < 0.01
+    assert stats.kstest(z, "norm").pvalue > 1e-3
+    # different seeds give different streams; same seed reproduces
+    assert np.array_equal(o.noise(42, 1000), z[:1000].astype(np.float32))
+    assert not np.array_equal(o.noise(43, 1000), o.noise(42, 1000))
+
+
+def test_box_muller_closed_form():
+    """u2 = 0 gives z = sqrt(-2 ln u1): check one element by hand from its words."""
+    seed = 7
+    n = np.arange(64, dtype=np.uint64)
+    w1 = o.splitmix64(np.uint64(seed) ^ o.splitmix64(np.uint64(2) * n))
+    w2 = o.splitmix64(np.uint64(seed) ^ o.splitmix64(np.uint64(2) * n + np.uint64(1)))
+    z = o.noise(seed, 64)
+    for i in (0, 17, 63):
+        u1 = ((int(w1[i]) >> 11) + 1) / 2.0 ** 53
+        u2 = (int(w2[i]) >> 11) / 2.0 ** 53
+        assert 0.0 < u1 <= 1.0 and 0.0 <= u2 < 1.0
+        assert z[i] == np.float32(math.sqrt(-2 * math.log(u1)) * math.cos(2 * math.pi * u2))
