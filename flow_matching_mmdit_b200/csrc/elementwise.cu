@@ -1,0 +1,373 @@
+// Memory-bound kernels of the denoiser path: seeded noise, patchify / unpatchify,
+// the RoPE table, RMSNorm + AdaLN modulation, the text-layer norm, the timestep
+// embedding MLP and the Euler / CFG update.  All accesses are coalesced (warp-per-row
+// or element-per-thread over the contiguous output), 128-bit where the row allows.
+#include <math.h>
+
+#include "kernels.cuh"
+
+namespace lens {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+inline int grid_for(int64_t n, int threads = kThreads) {
+  int64_t g = (n + threads - 1) / threads;
+  return (int)(g > (1 << 30) ? (1 << 30) : (g < 1 ? 1 : g));
+}
+
+// ---------------------------------------------------------------- noise
+// SplitMix64 output function at state v (Steele, Lea and Flood 2014; Vigna's
+// splitmix64.c): add the golden gamma, two xor-shift-multiply rounds, final shift.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t v) {
+  uint64_t z = v + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Standard normal for latent element n: Box-Muller on two SplitMix64 words,
+// u1 in (0, 1], u2 in [0, 1), evaluated in double and rounded to float.
+__device__ __forceinline__ float normal_at(uint64_t seed, uint64_t n) {
+  const uint64_t w1 = splitmix64(seed ^ splitmix64(2 * n));
+  const uint64_t w2 = splitmix64(seed ^ splitmix64(2 * n + 1));
+  const double u1 = (double)((w1 >> 11) + 1) * 0x1.0p-53;
+  const double u2 = (double)(w2 >> 11) * 0x1.0p-53;
+  return (float)(sqrt(-2.0 * log(u1)) * cos(2.0 * M_PI * u2));
+}
+
+// Token element e of [B, gh*gw, 128] <-> latent element of [B, 32, 2gh, 2gw]:
+// token (i, j) in row-major order, feature c*4 + 2r + s = latent[c, 2i + r, 2j + s].
+__device__ __forceinline__ int64_t latent_index_of_token(int64_t e, int gh, int gw) {
+  const int f = (int)(e & 127);
+  const int64_t tokb = e >> 7;
+  const int64_t ntok = (int64_t)gh * gw;
+  const int64_t b = tokb / ntok;
+  const int tok = (int)(tokb - b * ntok);
+  const int i = tok / gw, j = tok - (tok / gw) * gw;
+  const int c = f >> 2, r = (f >> 1) & 1, s = f & 1;
+  return (((b * kLatCh + c) * (2 * gh) + 2 * i + r) * (int64_t)(2 * gw)) + 2 * j + s;
+}
+
+__global__ void noise_tokens_kernel(uint64_t seed, int64_t n, int gh, int gw, float* __restrict__ tokens) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+    tokens[e] = normal_at(seed, (uint64_t)latent_index_of_token(e, gh, gw));
+}
+
+__global__ void patchify_kernel(const float* __restrict__ latent, int64_t n, int gh, int gw,
+                                float* __restrict__ tokens) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+    tokens[e] = latent[latent_index_of_token(e, gh, gw)];
+}
+
+__global__ void unpatchify_kernel(const float* __restrict__ tokens, int64_t n, int gh, int gw,
+                                  float* __restrict__ latent) {
+  const int W2 = 2 * gw, H2 = 2 * gh;
+  for (int64_t l = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; l < n; l += (int64_t)gridDim.x * blockDim.x) {
+    const int x = (int)(l % W2);
+    const int64_t r1 = l / W2;
+    const int y = (int)(r1 % H2);
+    const int64_t r2 = r1 / H2;
+    const int c = (int)(r2 % kLatCh);
+    const int64_t b = r2 / kLatCh;
+    const int64_t tok = b * gh * gw + (int64_t)(y >> 1) * gw + (x >> 1);
+    latent[l] = tokens[tok * kInCh + c * 4 + (y & 1) * 2 + (x & 1)];
+  }
+}
+
+// fp32 tokens -> bf16 GEMM operand [rows, 256] = [hi | lo], hi = bf16(x),
+// lo = bf16(x - hi), so the 128 -> 1536 projection sees x to ~16 bits.
+__global__ void tokens_to_operand_kernel(const float* __restrict__ tokens, int64_t n, int copies, int64_t copy_rows,
+                                         __nv_bfloat16* __restrict__ xin) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const float x = tokens[e];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+    const int64_t row = e >> 7;
+    const int f = (int)(e & 127);
+    for (int c = 0; c < copies; ++c) {
+      __nv_bfloat16* dst = xin + (row + c * copy_rows) * 256;
+      dst[f] = hi;
+      dst[128 + f] = lo;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- RoPE table
+// Pair p of the 64-dim head: p < 4 -> axis 0 (8 dims), p < 18 -> axis 1 (28 dims,
+// image row i), else axis 2 (28 dims, image column j).  Pair m of an axis of d_a
+// dims turns by pos * 10000^(-2m / d_a).  Text tokens (ids 0) get cos 1, sin 0.
+__global__ void rope_table_kernel(int gh, int gw, int n_txt, int ntok, float2* __restrict__ table) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= ntok * 32) return;
+  const int tok = e >> 5, p = e & 31;
+  int pos = 0, m, da;
+  if (p < 4) {
+    m = p;
+    da = 8;
+  } else if (p < 18) {
+    m = p - 4;
+    da = 28;
+    if (tok >= n_txt) pos = (tok - n_txt) / gw;
+  } else {
+    m = p - 18;
+    da = 28;
+    if (tok >= n_txt) pos = (tok - n_txt) % gw;
+  }
+  const double ang = (double)pos * pow(10000.0, -2.0 * m / (double)da);
+  table[e] = make_float2((float)cos(ang), (float)sin(ang));
+}
+
+// ---------------------------------------------------------------- RMSNorm + modulate
+// One warp per row of 1536 fp32: y = (1 + scale) * x * rsqrt(mean(x^2) + eps) + shift.
+__global__ void rmsnorm_modulate_kernel(const float* __restrict__ x, int M, int rows_per_batch,
+                                        const float* __restrict__ shift, const float* __restrict__ scale,
+                                        int64_t mod_stride, float eps, __nv_bfloat16* __restrict__ y) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)row * kHidden);
+  float4 v[12];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 12; ++i) {
+    v[i] = xr[lane + 32 * i];
+    ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = rsqrtf(ss * (1.0f / kHidden) + eps);
+  const int b = row / rows_per_batch;
+  const float4* sh = reinterpret_cast<const float4*>(shift + b * mod_stride);
+  const float4* sc = reinterpret_cast<const float4*>(scale + b * mod_stride);
+  uint2* yr = reinterpret_cast<uint2*>(y + (int64_t)row * kHidden);
+#pragma unroll
+  for (int i = 0; i < 12; ++i) {
+    const float4 a = __ldg(sh + lane + 32 * i), s = __ldg(sc + lane + 32 * i);
+    uint2 w;
+    w.x = pack_bf16x2((1.f + s.x) * v[i].x * r + a.x, (1.f + s.y) * v[i].y * r + a.y);
+    w.y = pack_bf16x2((1.f + s.z) * v[i].z * r + a.z, (1.f + s.w) * v[i].w * r + a.w);
+    yr[lane + 32 * i] = w;
+  }
+}
+
+// ---------------------------------------------------------------- text layers
+// One warp per (token, layer): RMSNorm of the 2880-wide slice times txt_norm.l,
+// written at column l * 2880 of the concatenated 11520-wide row.
+__global__ void text_norm_kernel(const __nv_bfloat16* __restrict__ E, int rows, const float* __restrict__ gains,
+                                 float eps, __nv_bfloat16* __restrict__ out) {
+  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (w >= rows * kTxtLayers) return;
+  const int layer = w % kTxtLayers;
+  const uint4* src = reinterpret_cast<const uint4*>(E + (int64_t)w * kTxtDim);
+  constexpr int kVec = kTxtDim / 8;   // 360
+  float ss = 0.f;
+  for (int i = lane; i < kVec; i += 32) {
+    const uint4 u = src[i];
+    const uint32_t p[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = bf16lo(p[j]), c = bf16hi(p[j]);
+      ss += a * a + c * c;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float r = rsqrtf(ss * (1.0f / kTxtDim) + eps);
+  const float* gl = gains + layer * kTxtDim;
+  uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)(w / kTxtLayers) * (kTxtLayers * kTxtDim) + layer * kTxtDim);
+  for (int i = lane; i < kVec; i += 32) {
+    const uint4 u = src[i];
+    const uint32_t p[4] = {u.x, u.y, u.z, u.w};
+    uint32_t q[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      q[j] = pack_bf16x2(bf16lo(p[j]) * r * __ldg(gl + 8 * i + 2 * j), bf16hi(p[j]) * r * __ldg(gl + 8 * i + 2 * j + 1));
+    dst[i] = make_uint4(q[0], q[1], q[2], q[3]);
+  }
+}
+
+// ---------------------------------------------------------------- timestep embedding
+// [cos(1000 t f_k) | sin(1000 t f_k)], f_k = exp(-ln(10000) k / 128), in double.
+__global__ void timestep_features_kernel(TimestepList tl, float* __restrict__ out) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= tl.T * kFreqDim) return;
+  const int ti = e / kFreqDim, k = e % kFreqDim;
+  const int half = kFreqDim / 2;
+  const int kk = k < half ? k : k - half;
+  const double f = exp(-log(10000.0) * (double)kk / (double)half);
+  const double a = 1000.0 * (double)tl.t[ti] * f;
+  out[e] = (float)(k < half ? cos(a) : sin(a));
+}
+
+// out[t][n] = sum_k W[n][k] * act(x[t][k]) + bias[n] for T <= 64 rows; act = SiLU or
+// identity.  One warp per output feature n, 8 rows of x staged in shared memory at a
+// time.  Optionally also writes bf16(SiLU(out)) and zero rows up to silu_rows (the
+// B operand of the modulation GEMM).
+__global__ void small_linear_kernel(const float* __restrict__ x, int T, int K, const __nv_bfloat16* __restrict__ W,
+                                    const float* __restrict__ bias, int N, int silu_in, float* __restrict__ out,
+                                    __nv_bfloat16* __restrict__ silu_out, int silu_rows) {
+  extern __shared__ float xs[];   // [8][K]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * (blockDim.x >> 5) + warp;
+  const __nv_bfloat16* wr = W + (int64_t)(n < N ? n : 0) * K;
+  for (int t0 = 0; t0 < T; t0 += 8) {
+    const int tc = min(8, T - t0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < tc * K; i += blockDim.x) {
+      float v = x[(int64_t)t0 * K + i];
+      if (silu_in) v = v / (1.f + expf(-v));
+      xs[i] = v;
+    }
+    __syncthreads();
+    float acc[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+    for (int k = lane * 8; k < K; k += 256) {
+      const uint4 u = *reinterpret_cast<const uint4*>(wr + k);
+      const uint32_t p[4] = {u.x, u.y, u.z, u.w};
+      float wv[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        wv[2 * j] = bf16lo(p[j]);
+        wv[2 * j + 1] = bf16hi(p[j]);
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if (r < tc) {
+          const float* xr = xs + r * K + k;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[r] += wv[j] * xr[j];
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      float a = acc[r];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0 && n < N && r < tc) {
+        const float y = a + (bias ? bias[n] : 0.f);
+        out[(int64_t)(t0 + r) * N + n] = y;
+        if (silu_out) silu_out[(int64_t)(t0 + r) * N + n] = __float2bfloat16_rn(y / (1.f + expf(-y)));
+      }
+    }
+  }
+  if (silu_out && lane == 0 && n < N)
+    for (int r = T; r < silu_rows; ++r) silu_out[(int64_t)r * N + n] = __float2bfloat16_rn(0.f);
+}
+
+// ---------------------------------------------------------------- Euler / CFG
+// x -= dt * v, v = vu + g (vc - vu) under CFG (v rows: B cond then B uncond) or vc.
+// Also refreshes the bf16 [hi | lo] operand of img_in for the next step (both the
+// cond and the uncond copy under CFG).
+__global__ void euler_cfg_kernel(float* __restrict__ x, const float* __restrict__ v, int64_t n, int64_t total_cond,
+                                 int cfg, float dt, float g, __nv_bfloat16* __restrict__ xin) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const float vc = v[e];
+    float vv = vc;
+    if (cfg) {
+      const float vu = v[total_cond + e];
+      vv = vu + g * (vc - vu);
+    }
+    const float xn = x[e] - dt * vv;
+    x[e] = xn;
+    if (xin) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(xn);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(xn - __bfloat162float(hi));
+      const int64_t row = e >> 7;
+      const int f = (int)(e & 127);
+      xin[row * 256 + f] = hi;
+      xin[row * 256 + 128 + f] = lo;
+      if (cfg) {
+        xin[(row + (total_cond >> 7)) * 256 + f] = hi;
+        xin[(row + (total_cond >> 7)) * 256 + 128 + f] = lo;
+      }
+    }
+  }
+}
+
+__global__ void euler_plain_kernel(float* __restrict__ x, const float* __restrict__ vc,
+                                   const float* __restrict__ vu, int64_t n, float dt, float g) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    float vv = vc[e];
+    if (vu) vv = vu[e] + g * (vv - vu[e]);
+    x[e] = x[e] - dt * vv;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_noise_tokens(uint64_t seed, int B, int gh, int gw, float* tokens, cudaStream_t st) {
+  const int64_t n = (int64_t)B * gh * gw * kInCh;
+  noise_tokens_kernel<<<grid_for(n), kThreads, 0, st>>>(seed, n, gh, gw, tokens);
+  return cudaGetLastError();
+}
+cudaError_t launch_patchify(const float* latent, int B, int gh, int gw, float* tokens, cudaStream_t st) {
+  const int64_t n = (int64_t)B * gh * gw * kInCh;
+  patchify_kernel<<<grid_for(n), kThreads, 0, st>>>(latent, n, gh, gw, tokens);
+  return cudaGetLastError();
+}
+cudaError_t launch_unpatchify(const float* tokens, int B, int gh, int gw, float* latent, cudaStream_t st) {
+  const int64_t n = (int64_t)B * gh * gw * kInCh;
+  unpatchify_kernel<<<grid_for(n), kThreads, 0, st>>>(tokens, n, gh, gw, latent);
+  return cudaGetLastError();
+}
+cudaError_t launch_tokens_to_operand(const float* tokens, int64_t rows, int copies, int64_t copy_rows,
+                                     __nv_bfloat16* xin, cudaStream_t st) {
+  const int64_t n = rows * kInCh;
+  tokens_to_operand_kernel<<<grid_for(n), kThreads, 0, st>>>(tokens, n, copies, copy_rows, xin);
+  return cudaGetLastError();
+}
+cudaError_t launch_rope_table(int gh, int gw, int n_txt, float2* table, cudaStream_t st) {
+  const int ntok = n_txt + gh * gw;
+  rope_table_kernel<<<grid_for((int64_t)ntok * 32), kThreads, 0, st>>>(gh, gw, n_txt, ntok, table);
+  return cudaGetLastError();
+}
+cudaError_t launch_rmsnorm_modulate(const float* x, int M, int rows_per_batch, const float* shift,
+                                    const float* scale, int64_t mod_stride, float eps, __nv_bfloat16* y,
+                                    cudaStream_t st) {
+  if (M <= 0) return cudaSuccess;
+  rmsnorm_modulate_kernel<<<(M + 7) / 8, 256, 0, st>>>(x, M, rows_per_batch, shift, scale, mod_stride, eps, y);
+  return cudaGetLastError();
+}
+cudaError_t launch_text_norm(const __nv_bfloat16* E, int rows, const float* gains, float eps, __nv_bfloat16* out,
+                             cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const int warps = rows * kTxtLayers;
+  text_norm_kernel<<<(warps + 7) / 8, 256, 0, st>>>(E, rows, gains, eps, out);
+  return cudaGetLastError();
+}
+cudaError_t launch_timestep_features(const TimestepList& tl, float* out, cudaStream_t st) {
+  timestep_features_kernel<<<grid_for((int64_t)tl.T * kFreqDim), kThreads, 0, st>>>(tl, out);
+  return cudaGetLastError();
+}
+cudaError_t launch_small_linear(const float* x, int T, int K, const __nv_bfloat16* W, const float* bias, int N,
+                                bool silu_in, float* out, __nv_bfloat16* silu_out_bf16, int silu_rows,
+                                cudaStream_t st) {
+  const size_t smem = (size_t)8 * K * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(small_linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  small_linear_kernel<<<(N + 7) / 8, 256, smem, st>>>(x, T, K, W, bias, N, silu_in ? 1 : 0, out, silu_out_bf16,
+                                                       silu_rows);
+  return cudaGetLastError();
+}
+cudaError_t launch_euler_cfg(float* x, const float* v, int64_t per_sample, int B, bool cfg, float dt,
+                             float guidance, __nv_bfloat16* xin, cudaStream_t st) {
+  const int64_t n = per_sample * B;
+  euler_cfg_kernel<<<grid_for(n), kThreads, 0, st>>>(x, v, n, n, cfg ? 1 : 0, dt, guidance, xin);
+  return cudaGetLastError();
+}
+cudaError_t launch_euler_plain(float* x, const float* vc, const float* vu, int64_t n, float dt, float guidance,
+                               cudaStream_t st) {
+  euler_plain_kernel<<<grid_for(n), kThreads, 0, st>>>(x, vc, vu, n, dt, guidance);
+  return cudaGetLastError();
+}
+
+}  // namespace lens

@@ -1,0 +1,96 @@
+// Host side of the tcgen05 GEMM: tensor-map encoding and the launch dispatcher.
+#include <mutex>
+
+#include "gemm.h"
+#include "gemm_tc.cuh"
+
+namespace lens {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+template <int BN, int EPI>
+cudaError_t launch_one(const CUtensorMap& A0, const CUtensorMap& B0, const CUtensorMap& A1, const CUtensorMap& B1,
+                       const GemmArgs& args, int sms, cudaStream_t st) {
+  using C = GemmCfg<BN>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = args.total_tiles < sms ? args.total_tiles : sms;
+  gemm_tc_kernel<BN, EPI><<<grid, 192, C::SMEM, st>>>(A0, B0, A1, B1, args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool encode_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
+                      uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || cols == 0) return false;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (row_stride_elems * 2) % 16 || box_rows == 0 || box_rows > 256)
+    return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride_elems * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+void finalize_problems(GemmArgs& a, int bn) {
+  int begin = 0;
+  for (int i = 0; i < a.num_problems; ++i) {
+    GemmProblem& p = a.p[i];
+    p.tiles_m = (p.M + 127) / 128;
+    p.tiles_n = (p.N + bn - 1) / bn;
+    p.tile_begin = begin;
+    begin += p.tiles_m * p.tiles_n;
+  }
+  a.total_tiles = begin;
+}
+
+cudaError_t launch_gemm(int bn, int epi, const CUtensorMap* A0, const CUtensorMap* B0, const CUtensorMap* A1,
+                        const CUtensorMap* B1, GemmArgs& args, int sms, cudaStream_t st) {
+  finalize_problems(args, bn);
+  if (args.total_tiles == 0) return cudaSuccess;
+  const CUtensorMap& a1 = A1 ? *A1 : *A0;
+  const CUtensorMap& b1 = B1 ? *B1 : *B0;
+#define LENS_GEMM_CASE(BN_, EPI_) \
+  if (bn == BN_ && epi == EPI_) return launch_one<BN_, EPI_>(*A0, *B0, a1, b1, args, sms, st);
+  LENS_GEMM_CASE(256, EPI_F32)
+  LENS_GEMM_CASE(128, EPI_F32)
+  LENS_GEMM_CASE(64, EPI_F32)
+  LENS_GEMM_CASE(32, EPI_F32)
+  LENS_GEMM_CASE(256, EPI_RESID)
+  LENS_GEMM_CASE(128, EPI_RESID)
+  LENS_GEMM_CASE(256, EPI_SWIGLU)
+  LENS_GEMM_CASE(256, EPI_QKV)
+  LENS_GEMM_CASE(16, EPI_F32_T)
+  LENS_GEMM_CASE(32, EPI_F32_T)
+  LENS_GEMM_CASE(64, EPI_F32_T)
+#undef LENS_GEMM_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lens

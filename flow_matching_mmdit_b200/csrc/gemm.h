@@ -1,0 +1,21 @@
+// Host interface of the tcgen05 GEMM (see gemm_tc.cuh for the kernel).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lens {
+
+struct GemmArgs;
+
+// 2D bf16 tensor map over a row-major [rows, cols] matrix (K = cols contiguous),
+// box = 64 columns x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+bool encode_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
+                      uint32_t box_rows);
+
+// Fill tile counts of args.p[0..num_problems) for tile width bn and launch the
+// persistent kernel (grid = min(tiles, sms)).  (bn, epi) must be an instantiated pair.
+cudaError_t launch_gemm(int bn, int epi, const CUtensorMap* A0, const CUtensorMap* B0, const CUtensorMap* A1,
+                        const CUtensorMap* B1, GemmArgs& args, int sms, cudaStream_t st);
+
+}  // namespace lens

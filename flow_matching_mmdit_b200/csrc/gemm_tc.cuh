@@ -1,0 +1,387 @@
+// Persistent tcgen05/TMEM GEMM for sm_100a with the denoiser's fused epilogues.
+//
+//   D[m, n] = sum_k A[m, k] * B[n, k]       A, B bf16, K-contiguous, fp32 accumulate
+//
+// One CTA per SM walks a static round-robin list of 128 x BN output tiles drawn
+// from up to two independent problems (the image and the text stream of a block
+// run as one launch).  Warp roles (192 threads):
+//   warp 0      TMA producer: 128x64 A and BNx64 B tiles, 128-byte swizzle,
+//               STAGES-deep ring of shared-memory stages
+//   warp 1      UMMA issuer (one thread): 4 x (M=128, N=BN, K=16) per stage into a
+//               TMEM accumulator; two accumulators so the epilogue of tile i
+//               overlaps the main loop of tile i+1
+//   warps 2..5  epilogue: each warp reads its 32 TMEM lanes (= 32 output rows),
+//               one row per thread, and applies the fused epilogue
+// Epilogues:
+//   EPI_F32     out = acc + bias                       (img_in, txt_in, proj_out)
+//   EPI_RESID   h  += gate[b] * (acc + bias)           (to_out / to_add_out, w2)
+//   EPI_SWIGLU  u   = silu(acc_g + b1) * (acc_u + b3)  (w1|w3 interleaved by 32)
+//   EPI_QKV     q, k: per-head RMSNorm * gain, RoPE; v as is; written head-major
+//               into the joint [B, 24, N, 64] sequence
+//   EPI_F32_T   out[n][m] = acc + bias[m]              (AdaLN modulation, A = weights)
+#pragma once
+#include "ptx.cuh"
+
+namespace lens {
+
+enum EpiKind { EPI_F32 = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3, EPI_F32_T = 4 };
+
+struct GemmProblem {
+  int M, N, K;
+  int tiles_m, tiles_n, tile_begin;
+  float* out_f32;
+  int64_t ld_out;
+  __nv_bfloat16* out_bf16;
+  const float* bias;
+  const float* gate;
+  int64_t gate_stride;
+  int rows_per_batch;
+  int n_valid;
+  __nv_bfloat16* q;
+  __nv_bfloat16* k;
+  __nv_bfloat16* v;
+  const float* gain_q;
+  const float* gain_k;
+  const float2* rope;
+  int n_tok;
+  int tok_offset;
+  int heads;
+  float eps;
+};
+
+struct GemmArgs {
+  GemmProblem p[2];
+  int num_problems;
+  int total_tiles;
+  int* err;
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (196608 / STAGE_BYTES) > 12 ? 12 : (196608 / STAGE_BYTES);
+  static constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
+  static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + 256;
+};
+
+__device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, int bn, int& pi, int& m0, int& n0) {
+  pi = (a.num_problems > 1 && t >= a.p[1].tile_begin) ? 1 : 0;
+  const GemmProblem& P = a.p[pi];
+  const int local = t - P.tile_begin;
+  m0 = (local % P.tiles_m) * 128;
+  n0 = (local / P.tiles_m) * bn;
+}
+
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+
+// ------------------------------------------------------------------ epilogues
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile(const GemmProblem& P, int row, int n0, uint32_t taddr) {
+  const bool live = row < P.M;
+  if constexpr (EPI == EPI_F32 || EPI == EPI_RESID) {
+    float* dst = P.out_f32 + (int64_t)row * P.ld_out + n0;
+    const float* gate = nullptr;
+    if constexpr (EPI == EPI_RESID) {
+      const int b = live ? row / P.rows_per_batch : 0;
+      gate = P.gate + (int64_t)b * P.gate_stride + n0;
+    }
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      float r[32];
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+      if (live) {
+        const int col = c * 32;
+        if (P.bias) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] += __ldg(P.bias + n0 + col + j);
+        }
+        float4* d4 = reinterpret_cast<float4*>(dst + col);
+        if constexpr (EPI == EPI_F32) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) d4[j] = make_float4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        } else {
+          const float4* g4 = reinterpret_cast<const float4*>(gate + col);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 h = d4[j];
+            const float4 g = __ldg(g4 + j);
+            h.x += g.x * r[4 * j];
+            h.y += g.y * r[4 * j + 1];
+            h.z += g.z * r[4 * j + 2];
+            h.w += g.w * r[4 * j + 3];
+            d4[j] = h;
+          }
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    // B rows were packed [w1 rows 32c..32c+31 | w3 rows 32c..32c+31] per 64 columns
+    __nv_bfloat16* dst = P.out_bf16 + (int64_t)row * (P.N / 2) + n0 / 2;
+#pragma unroll 1
+    for (int c = 0; c < BN / 64; ++c) {
+      float g[32], u[32];
+      tmem_ld32(taddr + c * 64, g);
+      tmem_ld32(taddr + c * 64 + 32, u);
+      tmem_ld_wait();
+      if (live) {
+        if (P.bias) {
+          const float* b = P.bias + n0 + c * 64;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            g[j] += __ldg(b + j);
+            u[j] += __ldg(b + 32 + j);
+          }
+        }
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 w;
+          w.x = pack_bf16x2(silu_f(g[8 * j + 0]) * u[8 * j + 0], silu_f(g[8 * j + 1]) * u[8 * j + 1]);
+          w.y = pack_bf16x2(silu_f(g[8 * j + 2]) * u[8 * j + 2], silu_f(g[8 * j + 3]) * u[8 * j + 3]);
+          w.z = pack_bf16x2(silu_f(g[8 * j + 4]) * u[8 * j + 4], silu_f(g[8 * j + 5]) * u[8 * j + 5]);
+          w.w = pack_bf16x2(silu_f(g[8 * j + 6]) * u[8 * j + 6], silu_f(g[8 * j + 7]) * u[8 * j + 7]);
+          d4[j] = w;
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_QKV) {
+    const int hidden = P.heads * 64;
+    const int sec = n0 / hidden;                  // 0 = q, 1 = k, 2 = v
+    const int head0 = (n0 - sec * hidden) / 64;
+    const int b = live ? row / P.rows_per_batch : 0;
+    const int tok = P.tok_offset + (live ? row - b * P.rows_per_batch : 0);
+    __nv_bfloat16* base = sec == 0 ? P.q : (sec == 1 ? P.k : P.v);
+    const float* gain = sec == 0 ? P.gain_q : P.gain_k;
+    const float2* rope = P.rope + (int64_t)tok * 32;
+#pragma unroll 1
+    for (int hh = 0; hh < BN / 64; ++hh) {
+      float x0[32], x1[32];
+      tmem_ld32(taddr + hh * 64, x0);
+      tmem_ld32(taddr + hh * 64 + 32, x1);
+      tmem_ld_wait();
+      if (!live) continue;
+      const int col = n0 + hh * 64;
+      if (P.bias) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          x0[j] += __ldg(P.bias + col + j);
+          x1[j] += __ldg(P.bias + col + 32 + j);
+        }
+      }
+      if (sec < 2) {
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ss += x0[j] * x0[j] + x1[j] * x1[j];
+        const float rs = rsqrtf(ss * (1.0f / 64.0f) + P.eps);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          x0[j] *= rs * __ldg(gain + j);
+          x1[j] *= rs * __ldg(gain + 32 + j);
+        }
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          const float2 cs = __ldg(rope + p);
+          const float a = x0[2 * p], bb = x0[2 * p + 1];
+          x0[2 * p] = a * cs.x - bb * cs.y;
+          x0[2 * p + 1] = a * cs.y + bb * cs.x;
+        }
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          const float2 cs = __ldg(rope + 16 + p);
+          const float a = x1[2 * p], bb = x1[2 * p + 1];
+          x1[2 * p] = a * cs.x - bb * cs.y;
+          x1[2 * p + 1] = a * cs.y + bb * cs.x;
+        }
+      }
+      const int head = head0 + hh;
+      uint4* d4 = reinterpret_cast<uint4*>(base + (((int64_t)b * P.heads + head) * P.n_tok + tok) * 64);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        d4[j] = make_uint4(pack_bf16x2(x0[8 * j], x0[8 * j + 1]), pack_bf16x2(x0[8 * j + 2], x0[8 * j + 3]),
+                           pack_bf16x2(x0[8 * j + 4], x0[8 * j + 5]), pack_bf16x2(x0[8 * j + 6], x0[8 * j + 7]));
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        d4[4 + j] = make_uint4(pack_bf16x2(x1[8 * j], x1[8 * j + 1]), pack_bf16x2(x1[8 * j + 2], x1[8 * j + 3]),
+                               pack_bf16x2(x1[8 * j + 4], x1[8 * j + 5]), pack_bf16x2(x1[8 * j + 6], x1[8 * j + 7]));
+    }
+  } else if constexpr (EPI == EPI_F32_T) {
+    const float bias = (live && P.bias) ? __ldg(P.bias + row) : 0.f;
+    if constexpr (BN == 16) {
+      float r[16];
+      tmem_ld16(taddr, r);
+      tmem_ld_wait();
+      if (live) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (n0 + j < P.n_valid) P.out_f32[(int64_t)(n0 + j) * P.ld_out + row] = r[j] + bias;
+      }
+    } else {
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float r[32];
+        tmem_ld32(taddr + c * 32, r);
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = n0 + c * 32 + j;
+            if (n < P.n_valid) P.out_f32[(int64_t)n * P.ld_out + row] = r[j] + bias;
+          }
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ GemmArgs args) {
+  using C = GemmCfg<BN>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmB0);
+    if (args.num_problems > 1) {
+      tma_prefetch_desc(&tmA1);
+      tma_prefetch_desc(&tmB1);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t last_parity[STAGES > 0 ? STAGES : 1];
+      bool issued[STAGES > 0 ? STAGES : 1];
+      for (int s = 0; s < STAGES; ++s) issued[s] = false, last_parity[s] = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < args.total_tiles && ok; t += gridDim.x) {
+        int pi, m0, n0;
+        decode_tile(args, t, BN, pi, m0, n0);
+        const CUtensorMap* mA = pi ? &tmA1 : &tmA0;
+        const CUtensorMap* mB = pi ? &tmB1 : &tmB0;
+        const int kblocks = args.p[pi].K / C::BK;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, args.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(sA + stage * C::A_BYTES, mA, &full[stage], kb * C::BK, m0);
+          tma_load_2d(sB + stage * C::B_BYTES, mB, &full[stage], kb * C::BK, n0);
+          issued[stage] = true;
+          last_parity[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // leave no copy in flight into this CTA's shared memory
+        for (int s = 0; s < STAGES; ++s)
+          if (issued[s]) mbar_wait_drain(&full[s], last_parity[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(128, BN);
+      uint32_t stage = 0, phase = 0;
+      int li = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < args.total_tiles && ok; t += gridDim.x, ++li) {
+        int pi, m0, n0;
+        decode_tile(args, t, BN, pi, m0, n0);
+        const int kblocks = args.p[pi].K / C::BK;
+        const uint32_t acc = li & 1;
+        const uint32_t use = li >> 1;
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, args.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
+          const uint64_t bd = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < C::BK / 16; ++k)
+            umma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int quarter = warp & 3;
+    int li = 0;
+    for (int t = blockIdx.x; t < args.total_tiles; t += gridDim.x, ++li) {
+      int pi, m0, n0;
+      decode_tile(args, t, BN, pi, m0, n0);
+      const uint32_t acc = li & 1;
+      const uint32_t use = li >> 1;
+      if (!mbar_wait(&tfull[acc], use & 1, args.err)) break;
+      tc_fence_after();
+      const int row = m0 + quarter * 32 + lane;
+      const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
+      epilogue_tile<BN, EPI>(args.p[pi], row, n0, taddr);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace lens

@@ -1,0 +1,56 @@
+// Declarations shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+
+namespace lens {
+
+constexpr int kHidden = 1536;
+constexpr int kHeads = 24;
+constexpr int kHeadDim = 64;
+constexpr int kMlp = 4096;
+constexpr int kInCh = 128;
+constexpr int kLatCh = 32;
+constexpr int kTxtLayers = 4;
+constexpr int kTxtDim = 2880;
+constexpr int kFreqDim = 256;
+constexpr int kModPerStream = 6 * kHidden;    // 9216
+constexpr int kModPerBlock = 2 * kModPerStream;
+constexpr int kMaxTimesteps = 64;             // per modulation launch (GEMM N <= 64)
+
+struct TimestepList {
+  float t[kMaxTimesteps];
+  int T;
+};
+
+// attention.cu
+cudaError_t launch_joint_attention(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int B,
+                                   int heads, int n_txt, int n_img, __nv_bfloat16* out_txt, __nv_bfloat16* out_img,
+                                   cudaStream_t st);
+
+// elementwise.cu
+cudaError_t launch_noise_tokens(uint64_t seed, int B, int gh, int gw, float* tokens, cudaStream_t st);
+cudaError_t launch_patchify(const float* latent, int B, int gh, int gw, float* tokens, cudaStream_t st);
+cudaError_t launch_unpatchify(const float* tokens, int B, int gh, int gw, float* latent, cudaStream_t st);
+cudaError_t launch_tokens_to_operand(const float* tokens, int64_t rows, int copies, int64_t copy_rows,
+                                     __nv_bfloat16* xin, cudaStream_t st);
+cudaError_t launch_rope_table(int gh, int gw, int n_txt, float2* table, cudaStream_t st);
+cudaError_t launch_rmsnorm_modulate(const float* x, int M, int rows_per_batch, const float* shift,
+                                    const float* scale, int64_t mod_stride, float eps, __nv_bfloat16* y,
+                                    cudaStream_t st);
+cudaError_t launch_text_norm(const __nv_bfloat16* E, int rows, const float* gains, float eps, __nv_bfloat16* out,
+                             cudaStream_t st);
+cudaError_t launch_timestep_features(const TimestepList& tl, float* out, cudaStream_t st);
+cudaError_t launch_small_linear(const float* x, int T, int K, const __nv_bfloat16* W, const float* bias, int N,
+                                bool silu_in, float* out, __nv_bfloat16* silu_out_bf16, int silu_rows,
+                                cudaStream_t st);
+cudaError_t launch_euler_cfg(float* x, const float* v, int64_t per_sample, int B, bool cfg, float dt,
+                             float guidance, __nv_bfloat16* xin, cudaStream_t st);
+cudaError_t launch_euler_plain(float* x, const float* vc, const float* vu, int64_t n, float dt, float guidance,
+                               cudaStream_t st);
+
+}  // namespace lens

@@ -1,0 +1,256 @@
+/*
+ * lens_dit.h — C ABI of the B200 (sm_100a) Lens MMDiT denoiser and its
+ * flow-matching Euler sampler.
+ *
+ * What is computed (sources are web pages, cited by title and section):
+ *   - "Lens" blog (zjwfufu.github.io), "Overview": 48 dual-stream MMDiT blocks,
+ *     hidden 1536, 24 heads, gated MLP 1536x4096, AdaLN 1536x9216 per stream.
+ *   - "深入 Lens-Turbo-3.8B-bf16 内核" (MLX bf16 port article), sections
+ *     "核心规格一览", "双流注意力机制", "自适应调制与 RMSNorm", "3D RoPE",
+ *     "多层级文本特征融合", "Patchify 补丁化与输出投影", "guidance 1.0": tensor
+ *     names, RoPE axes [8, 28, 28], 2x2 patches of a 32-channel latent (128-d
+ *     tokens), QK RMSNorm, four GPT-OSS feature layers of 2880.
+ *   - "Lens: 重新思考基础文生图模型的训练效率" (paper summary), "Flow Matching 训练目标":
+ *     x_t = (1-t) x0 + t x1, v = x1 - x0; "方法步骤详情": 20 steps with CFG 5.0,
+ *     Turbo 4 steps without CFG.
+ *   - "从提示词到成图：Lens-3.8B-4bit完整管线解析", section 6: pipeline(prompt,
+ *     height, width, num_inference_steps, seed); this ABI starts after the text
+ *     encoder (features in) and stops before the VAE (latent out).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers marked "dev" are caller-owned device memory on the current
+ *     device; "host" pointers are read during the call only.
+ *   - All GPU work is enqueued on `stream` (a cudaStream_t, NULL = legacy default
+ *     stream).  Argument errors return synchronously and enqueue nothing.  Errors
+ *     from kernels (including the device watchdog on internal waits) surface
+ *     through lens_dit_sync() or the next call.
+ *   - No entry point falls back to the CPU.  A handle is used by one stream at a
+ *     time.  Forward and sample calls allocate nothing: the handle's workspace is
+ *     sized at create time from the config's max_* fields.
+ *   - bf16 tensors are raw IEEE bfloat16 bit patterns (uint16_t here).
+ */
+#ifndef LENS_DIT_H
+#define LENS_DIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LENS_API __attribute__((visibility("default")))
+#else
+#define LENS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum lens_status {
+  LENS_OK = 0,
+  LENS_ERR_INVALID_ARG = 1,   /* null pointer, unknown tensor name, bad scalar */
+  LENS_ERR_SHAPE = 2,         /* shape out of range or inconsistent with the config */
+  LENS_ERR_OOM = 3,           /* device allocation failed at create */
+  LENS_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+  LENS_ERR_TIMEOUT = 5,       /* a kernel's bounded internal wait expired */
+  LENS_ERR_UNSUPPORTED = 6    /* config value this build does not implement */
+} lens_status;
+
+/* Model and capacity configuration.  Model fields must keep the Lens values
+ * (lens_dit_default_config); num_blocks may be 1..48 (fewer blocks run the first
+ * num_blocks of the tensor list, for tests).  max_* size the workspace:
+ * max_batch counts forward rows, i.e. 2 x samples when CFG is on. */
+typedef struct lens_dit_config {
+  int num_blocks;        /* 48 */
+  int hidden;            /* 1536 */
+  int heads;             /* 24 */
+  int head_dim;          /* 64 */
+  int mlp_hidden;        /* 4096 */
+  int in_channels;       /* 128 = 2*2*32 */
+  int latent_channels;   /* 32 */
+  int patch;             /* 2 */
+  int txt_layers;        /* 4 */
+  int txt_dim;           /* 2880 */
+  int rope_axes[3];      /* 8, 28, 28 */
+  float rope_theta;      /* 10000 */
+  float eps;             /* 1e-6, all RMSNorms */
+  int freq_dim;          /* 256, sinusoidal timestep features */
+  int max_batch;         /* forward rows (cond + uncond) */
+  int max_img_tokens;    /* grid_h * grid_w */
+  int max_txt_tokens;
+  int max_timesteps;     /* distinct timesteps whose modulation is kept at once */
+} lens_dit_config;
+
+/* One named weight tensor, host bf16, row-major [out, in] for Linear weights.
+ * Names (MLX bf16 port article, "双流注意力机制"/"自适应调制"/"多层级文本特征融合"):
+ *   time_text_embed.timestep_embedder.linear_{1,2}.{weight,bias}
+ *   txt_norm.{0..3}.weight, txt_in.{weight,bias}, img_in.{weight,bias}
+ *   transformer_blocks.{i}.{img_mod,txt_mod}.{weight,bias}
+ *   transformer_blocks.{i}.attn.{img_qkv,txt_qkv,to_out,to_add_out}.{weight,bias}
+ *   transformer_blocks.{i}.attn.{norm_q,norm_k,norm_added_q,norm_added_k}.weight
+ *   transformer_blocks.{i}.{img_mlp,txt_mlp}.{w1,w2,w3}.{weight,bias}
+ *   norm_out.linear.{weight,bias}, proj_out.{weight,bias}
+ * Every *.weight of a Linear is required; a missing bias is zero. */
+typedef struct lens_weight {
+  const char* name;
+  const uint16_t* data;   /* host bf16 */
+  int ndim;
+  int64_t shape[4];
+} lens_weight;
+
+typedef struct lens_dit lens_dit;
+
+/* Fill `cfg` with the Lens values and capacities for one 1024^2 CFG sample. */
+LENS_API lens_status lens_dit_default_config(lens_dit_config* cfg);
+
+/* Validate cfg, copy and pack the weights to the device (fused QKV as given,
+ * w1|w3 interleaved per 32 columns, all AdaLN projections and norm_out
+ * concatenated), and allocate the workspace.  The caller may free `w` on return.
+ * Synchronous.  Errors: INVALID_ARG (null, duplicate or unknown name, missing
+ * weight), SHAPE (a tensor shape differs from cfg), UNSUPPORTED (model fields
+ * other than Lens's), OOM, CUDA. */
+LENS_API lens_status lens_dit_create(const lens_dit_config* cfg, const lens_weight* w, int n_w,
+                            void* stream, lens_dit** out);
+
+LENS_API void lens_dit_destroy(lens_dit* h);
+
+/* One denoiser forward: velocity of B rows at per-row timesteps.
+ *   img_tokens  dev fp32 [B, grid_h*grid_w, 128]  patchified latent tokens
+ *   txt         dev bf16 [B, n_txt, 4, 2880]      encoder features of 4 layers
+ *   t           host fp32 [B]                     timesteps in [0, 1]
+ *   v_out       dev fp32 [B, grid_h*grid_w, 128]  velocity tokens
+ * Errors: INVALID_ARG (null), SHAPE (B > max_batch, B > max_timesteps, grid or
+ * n_txt beyond the capacities, n_txt + grid_h*grid_w < 1). */
+LENS_API lens_status lens_dit_forward(lens_dit* h, const float* img_tokens, int B, int grid_h, int grid_w,
+                             const uint16_t* txt, int n_txt, const float* t, float* v_out,
+                             void* stream);
+
+/* Flow-matching Euler sampler ("Flow Matching 训练目标": x_t = (1-t) x0 + t x1,
+ * v = x1 - x0; integrate t from 1 to 0 with `steps` uniform steps,
+ * x <- x - v / steps, model input t_k = 1 - k/steps).  With guidance != 1 the
+ * conditional and unconditional rows run as one batch of 2B and combine as
+ * uncond + guidance * (cond - uncond).
+ *   txt_cond    dev bf16 [B, n_txt, 4, 2880]
+ *   txt_uncond  dev bf16 [B, n_txt, 4, 2880], or NULL for zeros (ignored when
+ *               guidance == 1)
+ *   height_px, width_px: multiples of 16 (8x VAE, 2x2 patch)
+ *   seed        initial noise N(0,1): Box-Muller over SplitMix64 words, latent
+ *               element n uses words SM(seed ^ SM(2n)), SM(seed ^ SM(2n+1))
+ *   latent_out  dev fp32 [B, 32, height_px/8, width_px/8]
+ * Errors: INVALID_ARG (null, steps < 1, non-finite guidance), SHAPE (sizes not
+ * multiples of 16, beyond capacities, forward rows > max_batch). */
+LENS_API lens_status lens_sample_euler(lens_dit* h, const uint16_t* txt_cond, const uint16_t* txt_uncond,
+                              int B, int n_txt, int height_px, int width_px, int steps,
+                              float guidance, uint64_t seed, float* latent_out, void* stream);
+
+/* Test hook: run blocks [first, last) in place on a residual stream.
+ *   h_img dev fp32 [B, grid_h*grid_w, 1536], h_txt dev fp32 [B, n_txt, 1536]
+ *   t host fp32 [B].  Errors as lens_dit_forward, plus SHAPE for a bad range. */
+LENS_API lens_status lens_dit_debug_blocks(lens_dit* h, int first, int last, float* h_img, float* h_txt,
+                                  int B, int grid_h, int grid_w, int n_txt, const float* t,
+                                  void* stream);
+
+/* Wait for the handle's work on `stream` and report kernel-side errors
+ * (CUDA errors, TIMEOUT from the device watchdog).  Clears the watchdog flag. */
+LENS_API lens_status lens_dit_sync(lens_dit* h, void* stream);
+
+LENS_API const char* lens_status_string(lens_status s);
+
+/* ---------------------------------------------------------------------------
+ * Single-operation entry points (the same kernels the denoiser runs), for
+ * parity tests of each step.  Handle-free unless stated; no allocation.
+ * ------------------------------------------------------------------------- */
+
+/* Seeded N(0,1) latent noise straight into patch tokens (noise definition as in
+ * lens_sample_euler; patchify: token (i, j) of row-major order, feature
+ * c*4 + 2*r + s = latent[c, 2i+r, 2j+s]).  tokens dev fp32 [B, gh*gw, 128]. */
+LENS_API lens_status lens_op_noise_tokens(uint64_t seed, int B, int grid_h, int grid_w, float* tokens,
+                                 void* stream);
+
+/* Patchify a latent dev fp32 [B, 32, 2gh, 2gw] into tokens dev fp32
+ * [B, gh*gw, 128] and back (MLX port article, "Patchify 补丁化与输出投影").
+ * Bit-exact permutations. */
+LENS_API lens_status lens_op_patchify(const float* latent, int B, int grid_h, int grid_w, float* tokens,
+                             void* stream);
+LENS_API lens_status lens_op_unpatchify(const float* tokens, int B, int grid_h, int grid_w, float* latent,
+                               void* stream);
+
+/* 3D RoPE table (MLX port article, "3D RoPE"): ids (0,0,0) for the n_txt text
+ * tokens, then (0, i, j) for the image grid; pair m of axis a turns by
+ * pos_a * 10000^(-2m/d_a), axes [8, 28, 28] own consecutive head-dim segments.
+ * cos_sin dev fp32 [(n_txt + gh*gw), 32, 2] as (cos, sin) pairs. */
+LENS_API lens_status lens_op_rope_table(int grid_h, int grid_w, int n_txt, float* cos_sin, void* stream);
+
+/* y = (1 + scale[b]) * x / sqrt(mean(x^2) + eps) + shift[b] per row, rows of
+ * sample b = row / rows_per_batch ("自适应调制与 RMSNorm").
+ *   x dev fp32 [M, 1536]; shift, scale dev fp32 with row stride `mod_stride`
+ *   per sample; y dev bf16 [M, 1536]. */
+LENS_API lens_status lens_op_rmsnorm_modulate(const float* x, int M, int rows_per_batch,
+                                     const float* shift, const float* scale, int64_t mod_stride,
+                                     float eps, uint16_t* y, void* stream);
+
+/* Plain bf16 GEMM on the tcgen05 tensor cores: C[M,N] = A[M,K] B[N,K]^T (+ bias),
+ * fp32 out.  A, B dev bf16 K-contiguous; bias dev fp32 [N] or NULL; C dev fp32.
+ * K and N multiples of 64 and 16; A, B, C 16-byte aligned rows. */
+LENS_API lens_status lens_op_gemm_bf16(const uint16_t* A, const uint16_t* B, const float* bias, float* C,
+                              int M, int N, int K, void* stream);
+
+/* Joint attention over [text; image] tokens ("双流注意力机制"): per head
+ * softmax(q k^T / 8) v, no mask.  q, k, v dev bf16 [B, 24, N, 64] with
+ * N = n_txt + n_img, text rows first; out_txt dev bf16 [B, n_txt, 1536] and
+ * out_img dev bf16 [B, n_img, 1536] (column = head*64 + d). */
+LENS_API lens_status lens_op_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
+                              int n_txt, int n_img, uint16_t* out_txt, uint16_t* out_img,
+                              void* stream);
+
+/* Euler step with optional CFG on tokens: x -= dt * (vu + g (vc - vu)), or
+ * x -= dt * vc when v_uncond is NULL.  x, v_cond, v_uncond dev fp32 [n]. */
+LENS_API lens_status lens_op_euler_cfg(float* x, const float* v_cond, const float* v_uncond, int64_t n,
+                              float dt, float guidance, void* stream);
+
+/* Handle ops: the timestep embedding temb [T, 1536] (dev fp32) of host t[T], and
+ * the AdaLN modulation of every block plus norm_out for those timesteps,
+ * mod dev fp32 [T, 48*2*9216 + 3072] laid out block-major, then img/txt, then
+ * (shift1, scale1, gate1, shift2, scale2, gate2) x 1536; norm_out last as
+ * (scale, shift).  T <= max_timesteps. */
+LENS_API lens_status lens_dit_op_timestep(lens_dit* h, const float* t, int T, float* temb, float* mod,
+                                 void* stream);
+
+/* Handle op: text input head, txt dev bf16 [B, n_txt, 4, 2880] -> c dev fp32
+ * [B, n_txt, 1536] (txt_norm.0..3, concatenation, txt_in). */
+LENS_API lens_status lens_dit_op_text_input(lens_dit* h, const uint16_t* txt, int B, int n_txt, float* c,
+                                   void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Measurement hooks.
+ * ------------------------------------------------------------------------- */
+typedef enum lens_kernel {
+  LENS_KERNEL_NONE = 0,
+  LENS_KERNEL_ATTENTION = 1,     /* joint attention */
+  LENS_KERNEL_GEMM_QKV = 2,      /* QKV GEMM + QK-norm + RoPE epilogue */
+  LENS_KERNEL_GEMM_OUT = 3,      /* to_out / to_add_out GEMM + gated residual */
+  LENS_KERNEL_GEMM_W13 = 4,      /* w1|w3 GEMM + SwiGLU epilogue */
+  LENS_KERNEL_GEMM_W2 = 5,       /* w2 GEMM + gated residual */
+  LENS_KERNEL_RMSNORM_MOD = 6,   /* RMSNorm + AdaLN modulation */
+  LENS_KERNEL_GEMM_MOD = 7       /* all-block AdaLN modulation GEMM */
+} lens_kernel;
+
+/* Time every launch of one kernel family with a CUDA event pair recorded on the
+ * launching stream (up to `capacity` launches; later ones are not timed).
+ * kernel = LENS_KERNEL_NONE switches timing off.  Resets the record.  Creating
+ * the events is the only allocation; the call is synchronous. */
+LENS_API lens_status lens_dit_profile_kernel(lens_dit* h, lens_kernel kernel, int capacity);
+
+/* Synchronise the recorded events and report the timed launches and their summed
+ * device time in milliseconds. */
+LENS_API lens_status lens_dit_profile_read(lens_dit* h, int* launches, double* total_ms);
+
+/* Kernels this handle has launched since create (memcpy/memset not counted). */
+LENS_API int64_t lens_dit_launch_count(lens_dit* h);
+
+/* Number of streaming multiprocessors the kernels size their grids by. */
+LENS_API int lens_device_sm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LENS_DIT_H */

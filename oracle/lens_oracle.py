@@ -181,11 +181,15 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
     [survey] "交叉注意力与条件注入": text and image tokens are concatenated into one
     sequence for joint attention; [mlx] "双流注意力机制"."""
     d = q.shape[-1]
-    s = np.einsum("bhqd,bhkd->bhqk", q, k) / math.sqrt(d)
-    s = s - s.max(axis=-1, keepdims=True)
-    p = np.exp(s)
-    p = p / p.sum(axis=-1, keepdims=True)
-    return np.einsum("bhqk,bhkd->bhqd", p, v)
+    out = np.empty(q.shape[:-1] + (v.shape[-1],), dtype=np.result_type(q, v))
+    for b in range(q.shape[0]):                   # heads are independent; one at a time
+        for h in range(q.shape[1]):
+            s = (q[b, h] @ k[b, h].T) / math.sqrt(d)
+            s = s - s.max(axis=-1, keepdims=True)
+            p = np.exp(s)
+            p = p / p.sum(axis=-1, keepdims=True)
+            out[b, h] = p @ v[b, h]
+    return out
 
 
 # ============================================================ one dual-stream block (a6-a12)
