@@ -25,6 +25,7 @@ EXPORTS = [
     "lens_op_unpatchify", "lens_op_rope_table", "lens_op_rmsnorm_modulate", "lens_op_gemm_bf16",
     "lens_op_attention", "lens_op_euler_cfg", "lens_dit_op_timestep", "lens_dit_op_text_input",
     "lens_device_sm_count", "lens_dit_profile_kernel", "lens_dit_profile_read", "lens_dit_launch_count",
+    "lens_op_timestep_embed_noalloc",
 ]
 
 KERNELS = {"none": 0, "attention": 1, "gemm_qkv": 2, "gemm_out": 3, "gemm_w13": 4, "gemm_w2": 5, "rmsnorm_mod": 6,
@@ -87,6 +88,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lens_dit_profile_kernel": (I, [P, I, I]),
         "lens_dit_profile_read": (I, [P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]),
         "lens_dit_launch_count": (L, [P]),
+        "lens_op_timestep_embed_noalloc": (I, [P, I, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -265,6 +267,15 @@ def lens_dit_profile_read(h: LensDit):
 
 def lens_dit_launch_count(h: LensDit) -> int:
     return int(load_library().lens_dit_launch_count(h.ptr))
+
+
+def lens_op_timestep_embed_noalloc(t: Sequence[float], w1, b1, w2, b2, temb, stream=None) -> None:
+    """Timestep embedding for callers that cannot allocate device memory: all
+    intermediates stay in a fixed array inside the library (at most 64 timesteps)."""
+    tt = np.ascontiguousarray(np.asarray(t, np.float32))
+    _check(load_library().lens_op_timestep_embed_noalloc(tt.ctypes.data, len(tt), _ptr(w1), _ptr(b1), _ptr(w2),
+                                                         _ptr(b2), _ptr(temb), _stream(stream)),
+           "lens_op_timestep_embed_noalloc")
 
 
 def lens_device_sm_count() -> int:

@@ -220,6 +220,27 @@ LENS_API lens_status lens_dit_op_timestep(lens_dit* h, const float* t, int T, fl
 LENS_API lens_status lens_dit_op_text_input(lens_dit* h, const uint16_t* txt, int B, int n_txt, float* c,
                                    void* stream);
 
+/* Timestep embedding without any allocation.  The paper has no counterpart: this
+ * entry point exists for callers that cannot call cudaMalloc, for instance a plugin
+ * in a host application that owns and budgets all device memory, or a
+ * latency-critical loop that cannot afford cudaMalloc's implicit synchronisation.
+ * It computes the same temb as lens_dit_op_timestep (sinusoid -> linear_1 -> SiLU
+ * -> linear_2) from caller-supplied weights:
+ *   t     host fp32 [T], 1 <= T <= 64 (larger T returns LENS_ERR_SHAPE)
+ *   w1    dev bf16 [1536, 256],  b1 dev fp32 [1536] or NULL
+ *   w2    dev bf16 [1536, 1536], b2 dev fp32 [1536] or NULL
+ *   temb  dev fp32 [T, 1536]
+ * The intermediates live in one fixed 448 KiB device array inside the library,
+ * which every GPU that loads the library keeps until the process exits.  The first
+ * call on a device looks up that array's device address (with the device
+ * current); make that first call before any stream capture.  All calls share the
+ * array and it keeps the last call's contents (every value is written before it
+ * is read), so calls whose GPU work overlaps (e.g. on two streams at once) race.
+ * Calls no cudaMalloc, cudaFree or other allocating routine. */
+LENS_API lens_status lens_op_timestep_embed_noalloc(const float* t, int T, const uint16_t* w1, const float* b1,
+                                                    const uint16_t* w2, const float* b2, float* temb,
+                                                    void* stream);
+
 /* ---------------------------------------------------------------------------
  * Measurement hooks.
  * ------------------------------------------------------------------------- */
