@@ -58,6 +58,20 @@ bool encode_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t c
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || d0 == 0 || d1 == 0 || d2 == 0) return false;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (d0 * 2) % 16 || d0 * 2 > 128 || box_rows == 0 || box_rows > 256)
+    return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)d0, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 void finalize_problems(GemmArgs& a, int bn) {
   int begin = 0;
   for (int i = 0; i < a.num_problems; ++i) {

@@ -30,7 +30,7 @@ struct TimestepList {
 // attention.cu
 cudaError_t launch_joint_attention(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int B,
                                    int heads, int n_txt, int n_img, __nv_bfloat16* out_txt, __nv_bfloat16* out_img,
-                                   cudaStream_t st);
+                                   int* err, cudaStream_t st);
 
 // elementwise.cu
 cudaError_t launch_noise_tokens(uint64_t seed, int B, int gh, int gw, float* tokens, cudaStream_t st);

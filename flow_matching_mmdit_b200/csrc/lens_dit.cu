@@ -508,7 +508,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
     LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm(kBnQkv, EPI_QKV, &am.a_img, &wi.t_qkv, np > 1 ? &am.a_txt : nullptr,
                           np > 1 ? &wt.t_qkv : nullptr, a, h->sms, st));
   }
-  LENS_LAUNCH(h, LENS_KERNEL_ATTENTION, st, launch_joint_attention(h->q, h->k, h->v, B, kHeads, Nt, Ni, h->o_txt, h->o_img, st));
+  LENS_LAUNCH(h, LENS_KERNEL_ATTENTION, st, launch_joint_attention(h->q, h->k, h->v, B, kHeads, Nt, Ni, h->o_txt, h->o_img, h->err, st));
   {
     GemmArgs a = make_args(h->err);
     a.num_problems = np;
@@ -922,10 +922,14 @@ lens_status lens_op_attention(const uint16_t* q, const uint16_t* k, const uint16
                               uint16_t* out_txt, uint16_t* out_img, void* stream) {
   if (!q || !k || !v || (n_txt > 0 && !out_txt) || (n_img > 0 && !out_img)) return LENS_ERR_INVALID_ARG;
   if (B < 1 || n_txt < 0 || n_img < 0 || n_txt + n_img < 1) return LENS_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15)
+    return LENS_ERR_INVALID_ARG;
+  int* err = op_err_ptr();
+  if (!err) return LENS_ERR_CUDA;
   LENS_CUDA(launch_joint_attention(
       reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k),
       reinterpret_cast<const __nv_bfloat16*>(v), B, kHeads, n_txt, n_img, reinterpret_cast<__nv_bfloat16*>(out_txt),
-      reinterpret_cast<__nv_bfloat16*>(out_img), (cudaStream_t)stream));
+      reinterpret_cast<__nv_bfloat16*>(out_img), err, (cudaStream_t)stream));
   return LENS_OK;
 }
 

@@ -92,6 +92,21 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// 3D tiled load (x = innermost) completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy
+// (TMA, tensor cores).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
@@ -136,6 +151,12 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
          | (uint32_t(M >> 4) << 24);            // M / 16
 }
 
+// Instruction descriptor, kind::f16: bf16 A (K-major) and B (MN-major, i.e. N
+// contiguous per K row), fp32 D.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_bmn(int M, int N) {
+  return umma_idesc_bf16(M, N) | (1u << 16);
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile written by TMA with
 // 128-byte swizzle: rows of 64 bf16 (128 B), 8-row groups 1024 B apart.  The tile
 // base must be 1024-byte aligned; stepping K by 16 elements adds 32 B to the start.
@@ -143,6 +164,17 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
   return (uint64_t)((smem_addr & 0x3FFFFu) >> 4)      // start address
          | ((uint64_t)1 << 16)                        // leading byte offset (unused with SW128 K-major)
          | ((uint64_t)(1024 >> 4) << 32)              // stride byte offset: 8 rows x 128 B
+         | ((uint64_t)1 << 46)                        // descriptor version (sm_100)
+         | ((uint64_t)2 << 61);                       // swizzle: 128 B
+}
+
+// Descriptor for an MN-major operand written by TMA with 128-byte swizzle: each K
+// row holds 64 bf16 of N (128 B), 8-row K groups 1024 B apart.  N must be one
+// 64-element atom; stepping K by 16 adds 2048 B to the start.
+__device__ __forceinline__ uint64_t umma_desc_sw128_mn(uint32_t smem_addr) {
+  return (uint64_t)((smem_addr & 0x3FFFFu) >> 4)      // start address
+         | ((uint64_t)1 << 16)                        // leading byte offset (one atom along N: unused)
+         | ((uint64_t)(1024 >> 4) << 32)              // stride byte offset: 8 K rows x 128 B
          | ((uint64_t)1 << 46)                        // descriptor version (sm_100)
          | ((uint64_t)2 << 61);                       // swizzle: 128 B
 }
@@ -171,6 +203,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 32 consecutive fp32 columns from registers; thread i writes lane (base + i).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&r)[32]) {
+  const uint32_t* u = reinterpret_cast<const uint32_t*>(r);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]),
+      "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15]), "r"(u[16]), "r"(u[17]),
+      "r"(u[18]), "r"(u[19]), "r"(u[20]), "r"(u[21]), "r"(u[22]), "r"(u[23]), "r"(u[24]), "r"(u[25]), "r"(u[26]),
+      "r"(u[27]), "r"(u[28]), "r"(u[29]), "r"(u[30]), "r"(u[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t elect_lane0() { return (threadIdx.x & 31u) == 0u; }
 
