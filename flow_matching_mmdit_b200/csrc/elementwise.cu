@@ -121,13 +121,18 @@ __global__ void rope_table_kernel(int gh, int gw, int n_txt, int ntok, float2* _
 
 // ---------------------------------------------------------------- RMSNorm + modulate
 // One warp per row of 1536 fp32: y = (1 + scale) * x * rsqrt(mean(x^2) + eps) + shift.
-__global__ void rmsnorm_modulate_kernel(const float* __restrict__ x, int M, int rows_per_batch,
-                                        const float* __restrict__ shift, const float* __restrict__ scale,
-                                        int64_t mod_stride, float eps, __nv_bfloat16* __restrict__ y) {
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+// Up to two independent segments (the image and the text stream of a block) share
+// one launch: rows [0, s0.M) belong to segment 0, the next s1.M rows to segment 1.
+__global__ void rmsnorm_modulate_kernel(RmsSeg s0, RmsSeg s1, float eps) {
+  int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= M) return;
-  const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)row * kHidden);
+  const RmsSeg* sg = &s0;
+  if (row >= s0.M) {
+    row -= s0.M;
+    sg = &s1;
+    if (row >= s1.M) return;
+  }
+  const float4* xr = reinterpret_cast<const float4*>(sg->x + (int64_t)row * kHidden);
   float4 v[12];
   float ss = 0.f;
 #pragma unroll
@@ -138,10 +143,10 @@ __global__ void rmsnorm_modulate_kernel(const float* __restrict__ x, int M, int 
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float r = rsqrtf(ss * (1.0f / kHidden) + eps);
-  const int b = row / rows_per_batch;
-  const float4* sh = reinterpret_cast<const float4*>(shift + b * mod_stride);
-  const float4* sc = reinterpret_cast<const float4*>(scale + b * mod_stride);
-  uint2* yr = reinterpret_cast<uint2*>(y + (int64_t)row * kHidden);
+  const int b = row / sg->rows_per_batch;
+  const float4* sh = reinterpret_cast<const float4*>(sg->shift + b * sg->mod_stride);
+  const float4* sc = reinterpret_cast<const float4*>(sg->scale + b * sg->mod_stride);
+  uint2* yr = reinterpret_cast<uint2*>(sg->y + (int64_t)row * kHidden);
 #pragma unroll
   for (int i = 0; i < 12; ++i) {
     const float4 a = __ldg(sh + lane + 32 * i), s = __ldg(sc + lane + 32 * i);
@@ -326,12 +331,18 @@ cudaError_t launch_rope_table(int gh, int gw, int n_txt, float2* table, cudaStre
   rope_table_kernel<<<grid_for((int64_t)ntok * 32), kThreads, 0, st>>>(gh, gw, n_txt, ntok, table);
   return cudaGetLastError();
 }
+cudaError_t launch_rmsnorm_modulate(const RmsSeg& s0, const RmsSeg& s1, float eps, cudaStream_t st) {
+  const int M = s0.M + s1.M;
+  if (M <= 0) return cudaSuccess;
+  rmsnorm_modulate_kernel<<<(M + 7) / 8, 256, 0, st>>>(s0, s1, eps);
+  return cudaGetLastError();
+}
 cudaError_t launch_rmsnorm_modulate(const float* x, int M, int rows_per_batch, const float* shift,
                                     const float* scale, int64_t mod_stride, float eps, __nv_bfloat16* y,
                                     cudaStream_t st) {
-  if (M <= 0) return cudaSuccess;
-  rmsnorm_modulate_kernel<<<(M + 7) / 8, 256, 0, st>>>(x, M, rows_per_batch, shift, scale, mod_stride, eps, y);
-  return cudaGetLastError();
+  RmsSeg a{x, shift, scale, y, M, rows_per_batch, mod_stride};
+  RmsSeg none{x, shift, scale, y, 0, 1, 0};
+  return launch_rmsnorm_modulate(a, none, eps, st);
 }
 cudaError_t launch_text_norm(const __nv_bfloat16* E, int rows, const float* gains, float eps, __nv_bfloat16* out,
                              cudaStream_t st) {

@@ -27,8 +27,8 @@ EncodeTiledFn encode_fn() {
 
 template <int BN, int EPI>
 cudaError_t launch_one(const CUtensorMap& A0, const CUtensorMap& B0, const CUtensorMap& A1, const CUtensorMap& B1,
-                       const GemmArgs& args, int sms, cudaStream_t st) {
-  using C = GemmCfg<BN>;
+                       const CUtensorMap& C0, const CUtensorMap& C1, const GemmArgs& args, int sms, cudaStream_t st) {
+  using C = GemmCfg<BN, EPI>;
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -37,7 +37,7 @@ cudaError_t launch_one(const CUtensorMap& A0, const CUtensorMap& B0, const CUten
     attr = true;
   }
   const int grid = args.total_tiles < sms ? args.total_tiles : sms;
-  gemm_tc_kernel<BN, EPI><<<grid, 192, C::SMEM, st>>>(A0, B0, A1, B1, args);
+  gemm_tc_kernel<BN, EPI><<<grid, 192, C::SMEM, st>>>(A0, B0, A1, B1, C0, C1, args);
   return cudaGetLastError();
 }
 
@@ -55,6 +55,21 @@ bool encode_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t c
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_tmap_out(CUtensorMap* m, const void* ptr, int elem_bytes, uint64_t rows, uint64_t cols,
+                     uint64_t row_stride_elems) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || cols == 0 || (elem_bytes != 2 && elem_bytes != 4)) return false;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (row_stride_elems * elem_bytes) % 16) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride_elems * elem_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, elem_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -85,21 +100,29 @@ void finalize_problems(GemmArgs& a, int bn) {
 }
 
 cudaError_t launch_gemm(int bn, int epi, const CUtensorMap* A0, const CUtensorMap* B0, const CUtensorMap* A1,
-                        const CUtensorMap* B1, GemmArgs& args, int sms, cudaStream_t st) {
+                        const CUtensorMap* B1, const CUtensorMap* C0, const CUtensorMap* C1, GemmArgs& args, int sms,
+                        cudaStream_t st) {
   finalize_problems(args, bn);
   if (args.total_tiles == 0) return cudaSuccess;
+  if ((epi == EPI_F32 || epi == EPI_RESID || epi == EPI_SWIGLU) && (!C0 || (args.num_problems > 1 && !C1)))
+    return cudaErrorInvalidValue;
   const CUtensorMap& a1 = A1 ? *A1 : *A0;
   const CUtensorMap& b1 = B1 ? *B1 : *B0;
+  const CUtensorMap& c0 = C0 ? *C0 : *A0;
+  const CUtensorMap& c1 = C1 ? *C1 : c0;
 #define LENS_GEMM_CASE(BN_, EPI_) \
-  if (bn == BN_ && epi == EPI_) return launch_one<BN_, EPI_>(*A0, *B0, a1, b1, args, sms, st);
+  if (bn == BN_ && epi == EPI_) return launch_one<BN_, EPI_>(*A0, *B0, a1, b1, c0, c1, args, sms, st);
   LENS_GEMM_CASE(256, EPI_F32)
+  LENS_GEMM_CASE(192, EPI_F32)
   LENS_GEMM_CASE(128, EPI_F32)
   LENS_GEMM_CASE(64, EPI_F32)
   LENS_GEMM_CASE(32, EPI_F32)
   LENS_GEMM_CASE(256, EPI_RESID)
+  LENS_GEMM_CASE(192, EPI_RESID)
   LENS_GEMM_CASE(128, EPI_RESID)
   LENS_GEMM_CASE(256, EPI_SWIGLU)
   LENS_GEMM_CASE(256, EPI_QKV)
+  LENS_GEMM_CASE(192, EPI_QKV)
   LENS_GEMM_CASE(16, EPI_F32_T)
   LENS_GEMM_CASE(32, EPI_F32_T)
   LENS_GEMM_CASE(64, EPI_F32_T)

@@ -11,11 +11,14 @@
 //               TMEM accumulator; two accumulators so the epilogue of tile i
 //               overlaps the main loop of tile i+1
 //   warps 2..5  epilogue: each warp reads its 32 TMEM lanes (= 32 output rows),
-//               one row per thread, and applies the fused epilogue
+//               one row per thread, applies the fused epilogue, and (for the
+//               store kinds) stages 32 x 128-byte boxes in a double-buffered
+//               swizzled shared-memory slot that one lane ships with a TMA store
+//               or a TMA reduce-add
 // Epilogues:
-//   EPI_F32     out = acc + bias                       (img_in, txt_in, proj_out)
-//   EPI_RESID   h  += gate[b] * (acc + bias)           (to_out / to_add_out, w2)
-//   EPI_SWIGLU  u   = silu(acc_g + b1) * (acc_u + b3)  (w1|w3 interleaved by 32)
+//   EPI_F32     out = acc + bias                       (img_in, txt_in, proj_out)  TMA store
+//   EPI_RESID   h  += gate[b] * (acc + bias)           (to_out / to_add_out, w2)   TMA reduce-add
+//   EPI_SWIGLU  u   = silu(acc_g + b1) * (acc_u + b3)  (w1|w3 interleaved by 32)   TMA store
 //   EPI_QKV     q, k: per-head RMSNorm * gain, RoPE; v as is; written head-major
 //               into the joint [B, 24, N, 64] sequence
 //   EPI_F32_T   out[n][m] = acc + bias[m]              (AdaLN modulation, A = weights)
@@ -56,15 +59,26 @@ struct GemmArgs {
   int* err;
 };
 
-template <int BN>
+constexpr bool epi_uses_tma(int epi) { return epi == EPI_F32 || epi == EPI_RESID || epi == EPI_SWIGLU; }
+constexpr uint32_t pow2_at_least(uint32_t x) {
+  uint32_t p = 32;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+template <int BN, int EPI>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (196608 / STAGE_BYTES) > 12 ? 12 : (196608 / STAGE_BYTES);
-  static constexpr uint32_t TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
-  static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + 256;
+  // epilogue staging: 4 warps x 2 slots x (32 rows x 128 B)
+  static constexpr uint32_t EPI_SLOT = 4096;
+  static constexpr uint32_t EPI_BYTES = epi_uses_tma(EPI) ? 4 * 2 * EPI_SLOT : 0;
+  static constexpr uint32_t BUDGET = 232448 - 1024 - 256 - EPI_BYTES;
+  static constexpr int STAGES = (BUDGET / STAGE_BYTES) > 12 ? 12 : (BUDGET / STAGE_BYTES);
+  static constexpr uint32_t TMEM_COLS = pow2_at_least(2 * BN);
+  static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + 256;
 };
 
 __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, int bn, int& pi, int& m0, int& n0) {
@@ -78,11 +92,36 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, int bn, in
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
 
 // ------------------------------------------------------------------ epilogues
+// Stage one 32-row x 128-byte box (this thread's row = `lane`) in the warp's next
+// shared-memory slot with the 128-byte swizzle, then let lane 0 ship it.
+template <bool REDUCE>
+__device__ __forceinline__ void stage_and_ship(uint8_t* slots, uint32_t& slot, const uint4 (&chunk)[8],
+                                               const CUtensorMap* map, int x, int y, bool ship) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) bulk_wait_read<1>();          // the slot's previous box has been read out
+  __syncwarp();
+  uint8_t* buf = slots + slot * 4096;
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(buf + lane * 128 + ((c ^ (lane & 7)) << 4)) = chunk[c];
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0 && ship) {
+    if (REDUCE)
+      tma_reduce_add_2d(map, buf, x, y);
+    else
+      tma_store_2d(map, buf, x, y);
+  }
+  if (lane == 0) bulk_commit();
+  slot ^= 1;
+}
+
 template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_tile(const GemmProblem& P, int row, int n0, uint32_t taddr) {
+__device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtensorMap* tmC, int row, int row0_warp,
+                                              int n0, uint32_t taddr, uint8_t* slots, uint32_t& slot) {
   const bool live = row < P.M;
+  const bool any_live = row0_warp < P.M;
   if constexpr (EPI == EPI_F32 || EPI == EPI_RESID) {
-    float* dst = P.out_f32 + (int64_t)row * P.ld_out + n0;
     const float* gate = nullptr;
     if constexpr (EPI == EPI_RESID) {
       const int b = live ? row / P.rows_per_batch : 0;
@@ -93,60 +132,60 @@ __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, int row, int
       float r[32];
       tmem_ld32(taddr + c * 32, r);
       tmem_ld_wait();
-      if (live) {
-        const int col = c * 32;
-        if (P.bias) {
+      const int col = c * 32;
+      if (P.bias) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] += __ldg(P.bias + n0 + col + j);
-        }
-        float4* d4 = reinterpret_cast<float4*>(dst + col);
-        if constexpr (EPI == EPI_F32) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) d4[j] = make_float4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-        } else {
+        for (int j = 0; j < 32; ++j) r[j] += __ldg(P.bias + n0 + col + j);
+      }
+      if constexpr (EPI == EPI_RESID) {
+        if (live) {
           const float4* g4 = reinterpret_cast<const float4*>(gate + col);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            float4 h = d4[j];
             const float4 g = __ldg(g4 + j);
-            h.x += g.x * r[4 * j];
-            h.y += g.y * r[4 * j + 1];
-            h.z += g.z * r[4 * j + 2];
-            h.w += g.w * r[4 * j + 3];
-            d4[j] = h;
+            r[4 * j] *= g.x;
+            r[4 * j + 1] *= g.y;
+            r[4 * j + 2] *= g.z;
+            r[4 * j + 3] *= g.w;
           }
         }
       }
+      uint4 ch[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        ch[j] = make_uint4(__float_as_uint(r[4 * j]), __float_as_uint(r[4 * j + 1]), __float_as_uint(r[4 * j + 2]),
+                           __float_as_uint(r[4 * j + 3]));
+      stage_and_ship<EPI == EPI_RESID>(slots, slot, ch, tmC, n0 + col, row0_warp, any_live);
     }
   } else if constexpr (EPI == EPI_SWIGLU) {
-    // B rows were packed [w1 rows 32c..32c+31 | w3 rows 32c..32c+31] per 64 columns
-    __nv_bfloat16* dst = P.out_bf16 + (int64_t)row * (P.N / 2) + n0 / 2;
+    // B rows were packed [w1 rows 32c..32c+31 | w3 rows 32c..32c+31] per 64 columns;
+    // every 128 accumulator columns give 64 outputs = one 128-byte box row
 #pragma unroll 1
-    for (int c = 0; c < BN / 64; ++c) {
-      float g[32], u[32];
-      tmem_ld32(taddr + c * 64, g);
-      tmem_ld32(taddr + c * 64 + 32, u);
-      tmem_ld_wait();
-      if (live) {
+    for (int c = 0; c < BN / 128; ++c) {
+      uint4 ch[8];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float g[32], u[32];
+        tmem_ld32(taddr + c * 128 + half * 64, g);
+        tmem_ld32(taddr + c * 128 + half * 64 + 32, u);
+        tmem_ld_wait();
         if (P.bias) {
-          const float* b = P.bias + n0 + c * 64;
+          const float* b = P.bias + n0 + c * 128 + half * 64;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             g[j] += __ldg(b + j);
             u[j] += __ldg(b + 32 + j);
           }
         }
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 w;
-          w.x = pack_bf16x2(silu_f(g[8 * j + 0]) * u[8 * j + 0], silu_f(g[8 * j + 1]) * u[8 * j + 1]);
-          w.y = pack_bf16x2(silu_f(g[8 * j + 2]) * u[8 * j + 2], silu_f(g[8 * j + 3]) * u[8 * j + 3]);
-          w.z = pack_bf16x2(silu_f(g[8 * j + 4]) * u[8 * j + 4], silu_f(g[8 * j + 5]) * u[8 * j + 5]);
-          w.w = pack_bf16x2(silu_f(g[8 * j + 6]) * u[8 * j + 6], silu_f(g[8 * j + 7]) * u[8 * j + 7]);
-          d4[j] = w;
-        }
+        for (int j = 0; j < 4; ++j)
+          ch[half * 4 + j] =
+              make_uint4(pack_bf16x2(silu_f(g[8 * j + 0]) * u[8 * j + 0], silu_f(g[8 * j + 1]) * u[8 * j + 1]),
+                         pack_bf16x2(silu_f(g[8 * j + 2]) * u[8 * j + 2], silu_f(g[8 * j + 3]) * u[8 * j + 3]),
+                         pack_bf16x2(silu_f(g[8 * j + 4]) * u[8 * j + 4], silu_f(g[8 * j + 5]) * u[8 * j + 5]),
+                         pack_bf16x2(silu_f(g[8 * j + 6]) * u[8 * j + 6], silu_f(g[8 * j + 7]) * u[8 * j + 7]));
       }
+      stage_and_ship<false>(slots, slot, ch, tmC, n0 / 2 + c * 64, row0_warp, any_live);
     }
   } else if constexpr (EPI == EPI_QKV) {
     const int hidden = P.heads * 64;
@@ -242,14 +281,16 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1,
                    const __grid_constant__ GemmArgs args) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, EPI>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_BYTES);
+  uint8_t* sEpi = sB + STAGES * C::B_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + C::EPI_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -359,6 +400,8 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     const int quarter = warp & 3;
+    uint8_t* slots = sEpi + quarter * 2 * C::EPI_SLOT;
+    uint32_t slot = 0;
     int li = 0;
     for (int t = blockIdx.x; t < args.total_tiles; t += gridDim.x, ++li) {
       int pi, m0, n0;
@@ -367,12 +410,16 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t use = li >> 1;
       if (!mbar_wait(&tfull[acc], use & 1, args.err)) break;
       tc_fence_after();
-      const int row = m0 + quarter * 32 + lane;
+      const int row0 = m0 + quarter * 32;
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
-      epilogue_tile<BN, EPI>(args.p[pi], row, n0, taddr);
+      epilogue_tile<BN, EPI>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots, slot);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+    if constexpr (epi_uses_tma(EPI)) {
+      if (lane == 0) bulk_wait<0>();           // every box has landed before the CTA leaves
+      __syncwarp();
     }
   }
 

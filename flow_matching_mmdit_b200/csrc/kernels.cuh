@@ -39,6 +39,18 @@ cudaError_t launch_unpatchify(const float* tokens, int B, int gh, int gw, float*
 cudaError_t launch_tokens_to_operand(const float* tokens, int64_t rows, int copies, int64_t copy_rows,
                                      __nv_bfloat16* xin, cudaStream_t st);
 cudaError_t launch_rope_table(int gh, int gw, int n_txt, float2* table, cudaStream_t st);
+// One RMSNorm + modulate segment: rows of x [M, 1536] fp32 -> y bf16; sample b =
+// row / rows_per_batch reads shift / scale at b * mod_stride.
+struct RmsSeg {
+  const float* x;
+  const float* shift;
+  const float* scale;
+  __nv_bfloat16* y;
+  int M;
+  int rows_per_batch;
+  int64_t mod_stride;
+};
+cudaError_t launch_rmsnorm_modulate(const RmsSeg& s0, const RmsSeg& s1, float eps, cudaStream_t st);
 cudaError_t launch_rmsnorm_modulate(const float* x, int M, int rows_per_batch, const float* shift,
                                     const float* scale, int64_t mod_stride, float eps, __nv_bfloat16* y,
                                     cudaStream_t st);

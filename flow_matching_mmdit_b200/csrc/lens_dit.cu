@@ -20,7 +20,7 @@ using namespace lens;
 
 namespace {
 
-constexpr int kBnQkv = 256, kBnOut = 256, kBnW13 = 256, kBnW2 = 256, kBnImgIn = 256, kBnTxtIn = 128,
+constexpr int kBnQkv = 192, kBnOut = 192, kBnW13 = 256, kBnW2 = 192, kBnImgIn = 256, kBnTxtIn = 128,
               kBnProj = 128;
 
 struct StreamW {
@@ -424,7 +424,7 @@ static lens_status compute_modulation(lens_dit* h, const float* t, int T, cudaSt
   a.p[0].ld_out = h->modw;
   a.p[0].bias = h->b_mod;
   a.p[0].n_valid = T;
-  LENS_LAUNCH(h, LENS_KERNEL_GEMM_MOD, st, launch_gemm(Tpad, EPI_F32_T, &h->t_mod, &tb, nullptr, nullptr, a, h->sms, st));
+  LENS_LAUNCH(h, LENS_KERNEL_GEMM_MOD, st, launch_gemm(Tpad, EPI_F32_T, &h->t_mod, &tb, nullptr, nullptr, nullptr, nullptr, a, h->sms, st));
   return LENS_OK;
 }
 
@@ -442,8 +442,9 @@ static lens_status text_norm_rows(lens_dit* h, const uint16_t* txt, int rows, in
 
 static lens_status text_in_gemm(lens_dit* h, int rows, float* out, cudaStream_t st) {
   if (rows <= 0) return LENS_OK;
-  CUtensorMap ta;
-  if (!encode_tmap_bf16(&ta, h->txt_cat, rows, kTxtLayers * kTxtDim, kTxtLayers * kTxtDim, 128))
+  CUtensorMap ta, tc;
+  if (!encode_tmap_bf16(&ta, h->txt_cat, rows, kTxtLayers * kTxtDim, kTxtLayers * kTxtDim, 128) ||
+      !encode_tmap_out(&tc, out, 4, rows, kHidden, kHidden))
     return LENS_ERR_CUDA;
   GemmArgs a = make_args(h->err);
   a.num_problems = 1;
@@ -451,24 +452,31 @@ static lens_status text_in_gemm(lens_dit* h, int rows, float* out, cudaStream_t 
   a.p[0].out_f32 = out;
   a.p[0].ld_out = kHidden;
   a.p[0].bias = h->b_txt_in;
-  LENS_LAUNCH(h, 0, st, launch_gemm(kBnTxtIn, EPI_F32, &ta, &h->t_txt_in, nullptr, nullptr, a, h->sms, st));
+  LENS_LAUNCH(h, 0, st, launch_gemm(kBnTxtIn, EPI_F32, &ta, &h->t_txt_in, nullptr, nullptr, &tc, nullptr, a, h->sms, st));
   return LENS_OK;
 }
 
+// Tensor maps of one forward's activations: GEMM A operands (a, o, u as bf16, box
+// 128 rows) and TMA-store targets (residual streams h as fp32, u as bf16).
 struct ActMaps {
-  CUtensorMap a_img, a_txt, o_img, o_txt, u_img, u_txt;
+  CUtensorMap a_img, a_txt, o_img, o_txt, u_img, u_txt;      // A operands
+  CUtensorMap h_img, h_txt, uo_img, uo_txt;                  // epilogue outputs
   bool has_txt;
 };
 
-static lens_status make_act_maps(lens_dit* h, int Mi, int Mt, ActMaps& m) {
+static lens_status make_act_maps(lens_dit* h, int Mi, int Mt, float* hi, float* ht, ActMaps& m) {
   m.has_txt = Mt > 0;
   bool ok = encode_tmap_bf16(&m.a_img, h->a_img, Mi, kHidden, kHidden, 128) &&
             encode_tmap_bf16(&m.o_img, h->o_img, Mi, kHidden, kHidden, 128) &&
-            encode_tmap_bf16(&m.u_img, h->u_img, Mi, kMlp, kMlp, 128);
+            encode_tmap_bf16(&m.u_img, h->u_img, Mi, kMlp, kMlp, 128) &&
+            encode_tmap_out(&m.h_img, hi, 4, Mi, kHidden, kHidden) &&
+            encode_tmap_out(&m.uo_img, h->u_img, 2, Mi, kMlp, kMlp);
   if (m.has_txt)
     ok = ok && encode_tmap_bf16(&m.a_txt, h->a_txt, Mt, kHidden, kHidden, 128) &&
          encode_tmap_bf16(&m.o_txt, h->o_txt, Mt, kHidden, kHidden, 128) &&
-         encode_tmap_bf16(&m.u_txt, h->u_txt, Mt, kMlp, kMlp, 128);
+         encode_tmap_bf16(&m.u_txt, h->u_txt, Mt, kMlp, kMlp, 128) &&
+         encode_tmap_out(&m.h_txt, ht, 4, Mt, kHidden, kHidden) &&
+         encode_tmap_out(&m.uo_txt, h->u_txt, 2, Mt, kMlp, kMlp);
   return ok ? LENS_OK : LENS_ERR_CUDA;
 }
 
@@ -483,9 +491,12 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
   const StreamW& wt = h->blk[i].s[1];
   const int np = am.has_txt ? 2 : 1;
 
-  // attention branch
-  LENS_LAUNCH(h, LENS_KERNEL_RMSNORM_MOD, st, launch_rmsnorm_modulate(hi, Mi, Ni, mI, mI + kHidden, mstride, eps, h->a_img, st));
-  if (np > 1) LENS_LAUNCH(h, LENS_KERNEL_RMSNORM_MOD, st, launch_rmsnorm_modulate(ht, Mt, Nt, mT, mT + kHidden, mstride, eps, h->a_txt, st));
+  // attention branch (both streams in one launch)
+  {
+    const RmsSeg si{hi, mI, mI + kHidden, h->a_img, Mi, Ni, mstride};
+    const RmsSeg stx{ht, mT, mT + kHidden, h->a_txt, np > 1 ? Mt : 0, Nt > 0 ? Nt : 1, mstride};
+    LENS_LAUNCH(h, LENS_KERNEL_RMSNORM_MOD, st, launch_rmsnorm_modulate(si, stx, eps, st));
+  }
   {
     GemmArgs a = make_args(h->err);
     a.num_problems = np;
@@ -506,7 +517,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm(kBnQkv, EPI_QKV, &am.a_img, &wi.t_qkv, np > 1 ? &am.a_txt : nullptr,
-                          np > 1 ? &wt.t_qkv : nullptr, a, h->sms, st));
+                          np > 1 ? &wt.t_qkv : nullptr, nullptr, nullptr, a, h->sms, st));
   }
   LENS_LAUNCH(h, LENS_KERNEL_ATTENTION, st, launch_joint_attention(h->q, h->k, h->v, B, kHeads, Nt, Ni, h->o_txt, h->o_img, h->err, st));
   {
@@ -524,12 +535,14 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm(kBnOut, EPI_RESID, &am.o_img, &wi.t_out, np > 1 ? &am.o_txt : nullptr,
-                          np > 1 ? &wt.t_out : nullptr, a, h->sms, st));
+                          np > 1 ? &wt.t_out : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
   }
   // MLP branch
-  LENS_LAUNCH(h, LENS_KERNEL_RMSNORM_MOD, st, launch_rmsnorm_modulate(hi, Mi, Ni, mI + 3 * kHidden, mI + 4 * kHidden, mstride, eps, h->a_img, st));
-  if (np > 1)
-    LENS_LAUNCH(h, LENS_KERNEL_RMSNORM_MOD, st, launch_rmsnorm_modulate(ht, Mt, Nt, mT + 3 * kHidden, mT + 4 * kHidden, mstride, eps, h->a_txt, st));
+  {
+    const RmsSeg si{hi, mI + 3 * kHidden, mI + 4 * kHidden, h->a_img, Mi, Ni, mstride};
+    const RmsSeg stx{ht, mT + 3 * kHidden, mT + 4 * kHidden, h->a_txt, np > 1 ? Mt : 0, Nt > 0 ? Nt : 1, mstride};
+    LENS_LAUNCH(h, LENS_KERNEL_RMSNORM_MOD, st, launch_rmsnorm_modulate(si, stx, eps, st));
+  }
   {
     GemmArgs a = make_args(h->err);
     a.num_problems = np;
@@ -541,7 +554,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     LENS_LAUNCH(h, LENS_KERNEL_GEMM_W13, st, launch_gemm(kBnW13, EPI_SWIGLU, &am.a_img, &wi.t_w13, np > 1 ? &am.a_txt : nullptr,
-                          np > 1 ? &wt.t_w13 : nullptr, a, h->sms, st));
+                          np > 1 ? &wt.t_w13 : nullptr, &am.uo_img, np > 1 ? &am.uo_txt : nullptr, a, h->sms, st));
   }
   {
     GemmArgs a = make_args(h->err);
@@ -558,7 +571,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm(kBnW2, EPI_RESID, &am.u_img, &wi.t_w2, np > 1 ? &am.u_txt : nullptr,
-                          np > 1 ? &wt.t_w2 : nullptr, a, h->sms, st));
+                          np > 1 ? &wt.t_w2 : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
   }
   return LENS_OK;
 }
@@ -571,31 +584,35 @@ static lens_status run_forward_core(lens_dit* h, int B, int gh, int gw, int Nt, 
   lens_status s;
   LENS_LAUNCH(h, 0, st, launch_rope_table(gh, gw, Nt, h->rope, st));
   {
-    CUtensorMap tx;
-    if (!encode_tmap_bf16(&tx, h->xin, Mi, 2 * kInCh, 2 * kInCh, 128)) return LENS_ERR_CUDA;
+    CUtensorMap tx, th;
+    if (!encode_tmap_bf16(&tx, h->xin, Mi, 2 * kInCh, 2 * kInCh, 128) ||
+        !encode_tmap_out(&th, h->h_img, 4, Mi, kHidden, kHidden))
+      return LENS_ERR_CUDA;
     GemmArgs a = make_args(h->err);
     a.num_problems = 1;
     a.p[0] = base_problem(Mi, kHidden, 2 * kInCh);
     a.p[0].out_f32 = h->h_img;
     a.p[0].ld_out = kHidden;
     a.p[0].bias = h->b_img_in;
-    LENS_LAUNCH(h, 0, st, launch_gemm(kBnImgIn, EPI_F32, &tx, &h->t_img_in, nullptr, nullptr, a, h->sms, st));
+    LENS_LAUNCH(h, 0, st, launch_gemm(kBnImgIn, EPI_F32, &tx, &h->t_img_in, nullptr, nullptr, &th, nullptr, a, h->sms, st));
   }
   if (Mt > 0) LENS_CUDA(cudaMemcpyAsync(h->h_txt, h->h_txt0, (size_t)Mt * kHidden * 4, cudaMemcpyDeviceToDevice, st));
   ActMaps am;
-  if ((s = make_act_maps(h, Mi, Mt, am))) return s;
+  if ((s = make_act_maps(h, Mi, Mt, h->h_img, h->h_txt, am))) return s;
   for (int i = 0; i < h->cfg.num_blocks; ++i)
     if ((s = run_block(h, i, h->h_img, h->h_txt, B, Ni, Nt, mod, mstride, am, st))) return s;
   const float* no = mod + (int64_t)h->cfg.num_blocks * kModPerBlock;   // (scale, shift)
   LENS_LAUNCH(h, LENS_KERNEL_RMSNORM_MOD, st, launch_rmsnorm_modulate(h->h_img, Mi, Ni, no + kHidden, no, mstride, h->cfg.eps, h->a_img, st));
   {
+    CUtensorMap tv;
+    if (!encode_tmap_out(&tv, v_dst, 4, Mi, kInCh, kInCh)) return LENS_ERR_INVALID_ARG;
     GemmArgs a = make_args(h->err);
     a.num_problems = 1;
     a.p[0] = base_problem(Mi, kInCh, kHidden);
     a.p[0].out_f32 = v_dst;
     a.p[0].ld_out = kInCh;
     a.p[0].bias = h->b_proj;
-    LENS_LAUNCH(h, 0, st, launch_gemm(kBnProj, EPI_F32, &am.a_img, &h->t_proj, nullptr, nullptr, a, h->sms, st));
+    LENS_LAUNCH(h, 0, st, launch_gemm(kBnProj, EPI_F32, &am.a_img, &h->t_proj, nullptr, nullptr, &tv, nullptr, a, h->sms, st));
   }
   return LENS_OK;
 }
@@ -759,8 +776,9 @@ lens_status lens_dit_debug_blocks(lens_dit* h, int first, int last, float* h_img
   const int Ni = grid_h * grid_w;
   if ((s = compute_modulation(h, t, B, st))) return s;
   LENS_LAUNCH(h, 0, st, launch_rope_table(grid_h, grid_w, n_txt, h->rope, st));
+  if ((reinterpret_cast<uintptr_t>(h_img) | reinterpret_cast<uintptr_t>(h_txt)) & 15) return LENS_ERR_INVALID_ARG;
   ActMaps am;
-  if ((s = make_act_maps(h, B * Ni, B * n_txt, am))) return s;
+  if ((s = make_act_maps(h, B * Ni, B * n_txt, h_img, h_txt, am))) return s;
   for (int i = first; i < last; ++i)
     if ((s = run_block(h, i, h_img, h_txt, B, Ni, n_txt, h->mod, h->modw, am, st))) return s;
   return LENS_OK;
@@ -905,7 +923,8 @@ lens_status lens_op_gemm_bf16(const uint16_t* A, const uint16_t* Bm, const float
   CUtensorMap ta, tb;
   if (!encode_tmap_bf16(&ta, A, M, K, K, 128) || !encode_tmap_bf16(&tb, Bm, N, K, K, bn))
     return LENS_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(C) & 15) return LENS_ERR_INVALID_ARG;
+  CUtensorMap tc;
+  if (!encode_tmap_out(&tc, C, 4, M, N, N)) return LENS_ERR_INVALID_ARG;
   int* err = op_err_ptr();
   if (!err) return LENS_ERR_CUDA;
   GemmArgs a = make_args(err);
@@ -914,7 +933,7 @@ lens_status lens_op_gemm_bf16(const uint16_t* A, const uint16_t* Bm, const float
   a.p[0].out_f32 = C;
   a.p[0].ld_out = N;
   a.p[0].bias = bias;
-  LENS_CUDA(launch_gemm(bn, EPI_F32, &ta, &tb, nullptr, nullptr, a, device_sms(), (cudaStream_t)stream));
+  LENS_CUDA(launch_gemm(bn, EPI_F32, &ta, &tb, nullptr, nullptr, &tc, nullptr, a, device_sms(), (cudaStream_t)stream));
   return LENS_OK;
 }
 
