@@ -41,6 +41,23 @@ cudaError_t launch_one(const CUtensorMap& A0, const CUtensorMap& B0, const CUten
   return cudaGetLastError();
 }
 
+template <int BN, int EPI>
+cudaError_t launch_pair(const CUtensorMap& A0, const CUtensorMap& B0, const CUtensorMap& A1, const CUtensorMap& B1,
+                        const CUtensorMap& C0, const CUtensorMap& C1, const GemmArgs& args, int sms,
+                        cudaStream_t st) {
+  using C = Gemm2Cfg<BN, EPI>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(gemm2_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int pairs = args.total_tiles < sms / 2 ? args.total_tiles : sms / 2;
+  gemm2_tc_kernel<BN, EPI><<<2 * pairs, 192, C::SMEM, st>>>(A0, B0, A1, B1, C0, C1, args);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool encode_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
@@ -87,11 +104,11 @@ bool encode_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-void finalize_problems(GemmArgs& a, int bn) {
+void finalize_problems(GemmArgs& a, int bn, int bm) {
   int begin = 0;
   for (int i = 0; i < a.num_problems; ++i) {
     GemmProblem& p = a.p[i];
-    p.tiles_m = (p.M + 127) / 128;
+    p.tiles_m = (p.M + bm - 1) / bm;
     p.tiles_n = (p.N + bn - 1) / bn;
     p.tile_begin = begin;
     begin += p.tiles_m * p.tiles_n;
@@ -102,7 +119,7 @@ void finalize_problems(GemmArgs& a, int bn) {
 cudaError_t launch_gemm(int bn, int epi, const CUtensorMap* A0, const CUtensorMap* B0, const CUtensorMap* A1,
                         const CUtensorMap* B1, const CUtensorMap* C0, const CUtensorMap* C1, GemmArgs& args, int sms,
                         cudaStream_t st) {
-  finalize_problems(args, bn);
+  finalize_problems(args, bn, 128);
   if (args.total_tiles == 0) return cudaSuccess;
   if ((epi == EPI_F32 || epi == EPI_RESID || epi == EPI_SWIGLU) && (!C0 || (args.num_problems > 1 && !C1)))
     return cudaErrorInvalidValue;
@@ -127,6 +144,30 @@ cudaError_t launch_gemm(int bn, int epi, const CUtensorMap* A0, const CUtensorMa
   LENS_GEMM_CASE(32, EPI_F32_T)
   LENS_GEMM_CASE(64, EPI_F32_T)
 #undef LENS_GEMM_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm_pair(int bn, int epi, const CUtensorMap* A0, const CUtensorMap* B0, const CUtensorMap* A1,
+                             const CUtensorMap* B1, const CUtensorMap* C0, const CUtensorMap* C1, GemmArgs& args,
+                             int sms, cudaStream_t st) {
+  finalize_problems(args, bn, 256);
+  if (args.total_tiles == 0) return cudaSuccess;
+  if ((epi == EPI_F32 || epi == EPI_RESID || epi == EPI_SWIGLU) && (!C0 || (args.num_problems > 1 && !C1)))
+    return cudaErrorInvalidValue;
+  const CUtensorMap& a1 = A1 ? *A1 : *A0;
+  const CUtensorMap& b1 = B1 ? *B1 : *B0;
+  const CUtensorMap& c0 = C0 ? *C0 : *A0;
+  const CUtensorMap& c1 = C1 ? *C1 : c0;
+#define LENS_GEMM2_CASE(BN_, EPI_) \
+  if (bn == BN_ && epi == EPI_) return launch_pair<BN_, EPI_>(*A0, *B0, a1, b1, c0, c1, args, sms, st);
+  LENS_GEMM2_CASE(256, EPI_F32)
+  LENS_GEMM2_CASE(128, EPI_F32)
+  LENS_GEMM2_CASE(192, EPI_RESID)
+  LENS_GEMM2_CASE(256, EPI_RESID)
+  LENS_GEMM2_CASE(256, EPI_SWIGLU)
+  LENS_GEMM2_CASE(192, EPI_QKV)
+  LENS_GEMM2_CASE(256, EPI_QKV)
+#undef LENS_GEMM2_CASE
   return cudaErrorInvalidValue;
 }
 

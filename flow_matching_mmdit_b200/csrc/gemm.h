@@ -30,4 +30,10 @@ cudaError_t launch_gemm(int bn, int epi, const CUtensorMap* A0, const CUtensorMa
                         const CUtensorMap* B1, const CUtensorMap* C0, const CUtensorMap* C1, GemmArgs& args, int sms,
                         cudaStream_t st);
 
+// The same on 256 x bn tiles computed by CTA pairs (cta_group::2): A maps keep a box
+// of 128 rows, B maps need a box of bn / 2 rows.  Grid = 2 x min(tiles, sms / 2).
+cudaError_t launch_gemm_pair(int bn, int epi, const CUtensorMap* A0, const CUtensorMap* B0, const CUtensorMap* A1,
+                             const CUtensorMap* B1, const CUtensorMap* C0, const CUtensorMap* C1, GemmArgs& args,
+                             int sms, cudaStream_t st);
+
 }  // namespace lens

@@ -75,10 +75,11 @@ struct GemmCfg {
   // epilogue staging: 4 warps x 2 slots x (32 rows x 128 B)
   static constexpr uint32_t EPI_SLOT = 4096;
   static constexpr uint32_t EPI_BYTES = epi_uses_tma(EPI) ? 4 * 2 * EPI_SLOT : 0;
-  static constexpr uint32_t BUDGET = 232448 - 1024 - 256 - EPI_BYTES;
+  static constexpr uint32_t AUX_BYTES = EPI == EPI_QKV ? 1024 : 0;
+  static constexpr uint32_t BUDGET = 232448 - 1024 - 256 - EPI_BYTES - AUX_BYTES;
   static constexpr int STAGES = (BUDGET / STAGE_BYTES) > 12 ? 12 : (BUDGET / STAGE_BYTES);
   static constexpr uint32_t TMEM_COLS = pow2_at_least(2 * BN);
-  static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + 256;
+  static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + AUX_BYTES + 256;
 };
 
 __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, int bn, int& pi, int& m0, int& n0) {
@@ -118,7 +119,8 @@ __device__ __forceinline__ void stage_and_ship(uint8_t* slots, uint32_t& slot, c
 
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtensorMap* tmC, int row, int row0_warp,
-                                              int n0, uint32_t taddr, uint8_t* slots, uint32_t& slot) {
+                                              int n0, uint32_t taddr, uint8_t* slots, uint32_t& slot,
+                                              const float* qk_gains) {
   const bool live = row < P.M;
   const bool any_live = row0_warp < P.M;
   if constexpr (EPI == EPI_F32 || EPI == EPI_RESID) {
@@ -188,64 +190,63 @@ __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtens
       stage_and_ship<false>(slots, slot, ch, tmC, n0 / 2 + c * 64, row0_warp, any_live);
     }
   } else if constexpr (EPI == EPI_QKV) {
+    // gains: the problem's q and k gains staged in shared memory at kernel start
     const int hidden = P.heads * 64;
     const int sec = n0 / hidden;                  // 0 = q, 1 = k, 2 = v
     const int head0 = (n0 - sec * hidden) / 64;
     const int b = live ? row / P.rows_per_batch : 0;
     const int tok = P.tok_offset + (live ? row - b * P.rows_per_batch : 0);
     __nv_bfloat16* base = sec == 0 ? P.q : (sec == 1 ? P.k : P.v);
-    const float* gain = sec == 0 ? P.gain_q : P.gain_k;
-    const float2* rope = P.rope + (int64_t)tok * 32;
+    const float4* gain4 = reinterpret_cast<const float4*>(qk_gains + (sec == 0 ? 0 : 64));
+    float4 rp[16];                                // this row's (cos, sin) pairs, once per tile
+    if (sec < 2 && live) {
+      const float4* rope4 = reinterpret_cast<const float4*>(P.rope + (int64_t)tok * 32);
+#pragma unroll
+      for (int p = 0; p < 16; ++p) rp[p] = __ldg(rope4 + p);
+    }
 #pragma unroll 1
     for (int hh = 0; hh < BN / 64; ++hh) {
-      float x0[32], x1[32];
-      tmem_ld32(taddr + hh * 64, x0);
-      tmem_ld32(taddr + hh * 64 + 32, x1);
+      float x[64];
+      tmem_ld32(taddr + hh * 64, *reinterpret_cast<float(*)[32]>(&x[0]));
+      tmem_ld32(taddr + hh * 64 + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
       tmem_ld_wait();
       if (!live) continue;
       const int col = n0 + hh * 64;
       if (P.bias) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          x0[j] += __ldg(P.bias + col + j);
-          x1[j] += __ldg(P.bias + col + 32 + j);
-        }
+        for (int j = 0; j < 64; ++j) x[j] += __ldg(P.bias + col + j);
       }
       if (sec < 2) {
-        float ss = 0.f;
+        float ss0 = 0.f, ss1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) ss += x0[j] * x0[j] + x1[j] * x1[j];
-        const float rs = rsqrtf(ss * (1.0f / 64.0f) + P.eps);
+        for (int j = 0; j < 64; j += 2) {
+          ss0 += x[j] * x[j];
+          ss1 += x[j + 1] * x[j + 1];
+        }
+        const float rs = rsqrtf((ss0 + ss1) * (1.0f / 64.0f) + P.eps);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          x0[j] *= rs * __ldg(gain + j);
-          x1[j] *= rs * __ldg(gain + 32 + j);
+        for (int q4 = 0; q4 < 16; ++q4) {
+          const float4 g = gain4[q4];
+          x[4 * q4] *= rs * g.x;
+          x[4 * q4 + 1] *= rs * g.y;
+          x[4 * q4 + 2] *= rs * g.z;
+          x[4 * q4 + 3] *= rs * g.w;
         }
 #pragma unroll
-        for (int p = 0; p < 16; ++p) {
-          const float2 cs = __ldg(rope + p);
-          const float a = x0[2 * p], bb = x0[2 * p + 1];
-          x0[2 * p] = a * cs.x - bb * cs.y;
-          x0[2 * p + 1] = a * cs.y + bb * cs.x;
-        }
-#pragma unroll
-        for (int p = 0; p < 16; ++p) {
-          const float2 cs = __ldg(rope + 16 + p);
-          const float a = x1[2 * p], bb = x1[2 * p + 1];
-          x1[2 * p] = a * cs.x - bb * cs.y;
-          x1[2 * p + 1] = a * cs.y + bb * cs.x;
+        for (int p = 0; p < 16; ++p) {           // pairs 2p and 2p+1 of rp[p]
+          const float a0 = x[4 * p], b0 = x[4 * p + 1], a1 = x[4 * p + 2], b1 = x[4 * p + 3];
+          x[4 * p] = a0 * rp[p].x - b0 * rp[p].y;
+          x[4 * p + 1] = a0 * rp[p].y + b0 * rp[p].x;
+          x[4 * p + 2] = a1 * rp[p].z - b1 * rp[p].w;
+          x[4 * p + 3] = a1 * rp[p].w + b1 * rp[p].z;
         }
       }
       const int head = head0 + hh;
       uint4* d4 = reinterpret_cast<uint4*>(base + (((int64_t)b * P.heads + head) * P.n_tok + tok) * 64);
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        d4[j] = make_uint4(pack_bf16x2(x0[8 * j], x0[8 * j + 1]), pack_bf16x2(x0[8 * j + 2], x0[8 * j + 3]),
-                           pack_bf16x2(x0[8 * j + 4], x0[8 * j + 5]), pack_bf16x2(x0[8 * j + 6], x0[8 * j + 7]));
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        d4[4 + j] = make_uint4(pack_bf16x2(x1[8 * j], x1[8 * j + 1]), pack_bf16x2(x1[8 * j + 2], x1[8 * j + 3]),
-                               pack_bf16x2(x1[8 * j + 4], x1[8 * j + 5]), pack_bf16x2(x1[8 * j + 6], x1[8 * j + 7]));
+      for (int j = 0; j < 8; ++j)
+        d4[j] = make_uint4(pack_bf16x2(x[8 * j], x[8 * j + 1]), pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
+                           pack_bf16x2(x[8 * j + 4], x[8 * j + 5]), pack_bf16x2(x[8 * j + 6], x[8 * j + 7]));
     }
   } else if constexpr (EPI == EPI_F32_T) {
     const float bias = (live && P.bias) ? __ldg(P.bias + row) : 0.f;
@@ -290,7 +291,8 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * C::A_BYTES;
   uint8_t* sEpi = sB + STAGES * C::B_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + C::EPI_BYTES);
+  float* sAux = reinterpret_cast<float*>(sEpi + C::EPI_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + C::EPI_BYTES + C::AUX_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -314,6 +316,12 @@ __global__ void __launch_bounds__(192, 1)
     if (args.num_problems > 1) {
       tma_prefetch_desc(&tmA1);
       tma_prefetch_desc(&tmB1);
+    }
+  }
+  if constexpr (EPI == EPI_QKV) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+      const GemmProblem& P = args.p[(i >> 7) < args.num_problems ? (i >> 7) : 0];
+      sAux[i] = (i & 64) ? P.gain_k[i & 63] : P.gain_q[i & 63];
     }
   }
   if (warp == 1) {
@@ -412,7 +420,8 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int row0 = m0 + quarter * 32;
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
-      epilogue_tile<BN, EPI>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots, slot);
+      epilogue_tile<BN, EPI>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots, slot,
+                             sAux + pi * 128);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -428,6 +437,204 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ==================================================================== CTA-pair version
+// The same problem list and epilogues on 256 x BN tiles computed by a cluster of two
+// CTAs with cta_group::2 UMMA: CTA rank r stages A rows [m0 + 128 r, +128) and B
+// rows [n0 + r BN/2, +BN/2); the leader (rank 0) issues M = 256 MMAs that read both
+// CTAs' shared memory and write each CTA's 128-row half of D into its own TMEM.
+// Per output element this halves the B operand traffic into shared memory.
+//   full[s]    (leader)  TMA bytes of both CTAs; armed by the leader's producer
+//   empty[s]   (both)    MMA commit multicast: stage s may be refilled
+//   tfull[a]   (both)    MMA commit multicast: accumulator a holds a finished tile
+//   tempty[a]  (leader)  8 arrivals (4 epilogue warps x 2 CTAs): accumulator a free
+template <int BN, int EPI>
+struct Gemm2Cfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = (BN / 2) * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t EPI_SLOT = 4096;
+  static constexpr uint32_t EPI_BYTES = epi_uses_tma(EPI) ? 4 * 2 * EPI_SLOT : 0;
+  static constexpr uint32_t AUX_BYTES = EPI == EPI_QKV ? 1024 : 0;
+  static constexpr uint32_t BUDGET = 232448 - 1024 - 256 - EPI_BYTES - AUX_BYTES;
+  static constexpr int STAGES = (BUDGET / STAGE_BYTES) > 8 ? 8 : (BUDGET / STAGE_BYTES);
+  static constexpr uint32_t TMEM_COLS = pow2_at_least(2 * BN);
+  static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + AUX_BYTES + 256;
+};
+
+__device__ __forceinline__ void decode_tile2(const GemmArgs& a, int t, int bn, int& pi, int& m0, int& n0) {
+  pi = (a.num_problems > 1 && t >= a.p[1].tile_begin) ? 1 : 0;
+  const GemmProblem& P = a.p[pi];
+  const int local = t - P.tile_begin;
+  m0 = (local % P.tiles_m) * 256;
+  n0 = (local / P.tiles_m) * bn;
+}
+
+template <int BN, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    gemm2_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                    const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1,
+                    const __grid_constant__ GemmArgs args) {
+  using C = Gemm2Cfg<BN, EPI>;
+  constexpr int STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * C::A_BYTES;
+  uint8_t* sEpi = sB + STAGES * C::B_BYTES;
+  float* sAux = reinterpret_cast<float*>(sEpi + C::EPI_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + C::EPI_BYTES + C::AUX_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 8);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmB0);
+    if (args.num_problems > 1) {
+      tma_prefetch_desc(&tmA1);
+      tma_prefetch_desc(&tmB1);
+    }
+  }
+  if constexpr (EPI == EPI_QKV) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+      const GemmProblem& P = args.p[(i >> 7) < args.num_problems ? (i >> 7) : 0];
+      sAux[i] = (i & 64) ? P.gain_k[i & 63] : P.gain_q[i & 63];
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();          // both CTAs' barriers initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t last_parity[STAGES];
+      bool issued[STAGES];
+      for (int s = 0; s < STAGES; ++s) issued[s] = false, last_parity[s] = 0;
+      bool ok = true;
+      for (int t = pair; t < args.total_tiles && ok; t += npairs) {
+        int pi, m0, n0;
+        decode_tile2(args, t, BN, pi, m0, n0);
+        const CUtensorMap* mA = pi ? &tmA1 : &tmA0;
+        const CUtensorMap* mB = pi ? &tmB1 : &tmB0;
+        const int kblocks = args.p[pi].K / C::BK;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, args.err)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          tma_load_2d_pair(sA + stage * C::A_BYTES, mA, &full[stage], kb * C::BK, m0 + 128 * (int)rank);
+          tma_load_2d_pair(sB + stage * C::B_BYTES, mB, &full[stage], kb * C::BK, n0 + (BN / 2) * (int)rank);
+          issued[stage] = true;
+          last_parity[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && rank == 0) {
+        for (int s = 0; s < STAGES; ++s)
+          if (issued[s]) mbar_wait_drain(&full[s], last_parity[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(256, BN);
+      uint32_t stage = 0, phase = 0;
+      int li = 0;
+      bool ok = true;
+      for (int t = pair; t < args.total_tiles && ok; t += npairs, ++li) {
+        int pi, m0, n0;
+        decode_tile2(args, t, BN, pi, m0, n0);
+        const int kblocks = args.p[pi].K / C::BK;
+        const uint32_t acc = li & 1;
+        const uint32_t use = li >> 1;
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, args.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
+          const uint64_t bd = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < C::BK / 16; ++k)
+            umma_bf16_pair(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair(&empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(&tfull[acc], 0x3);
+      }
+    }
+    __syncwarp();
+  } else {
+    const int quarter = warp & 3;
+    uint8_t* slots = sEpi + quarter * 2 * C::EPI_SLOT;
+    uint32_t slot = 0;
+    const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    int li = 0;
+    for (int t = pair; t < args.total_tiles; t += npairs, ++li) {
+      int pi, m0, n0;
+      decode_tile2(args, t, BN, pi, m0, n0);
+      const uint32_t acc = li & 1;
+      const uint32_t use = li >> 1;
+      if (!mbar_wait(&tfull[acc], use & 1, args.err)) break;
+      tc_fence_after();
+      const int row0 = m0 + 128 * (int)rank + quarter * 32;
+      const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
+      epilogue_tile<BN, EPI>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots, slot,
+                             sAux + pi * 128);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tempty0 + acc * 8);
+    }
+    if constexpr (epi_uses_tma(EPI)) {
+      if (lane == 0) bulk_wait<0>();
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();          // no MMA, TMA or remote arrive of the pair is still in flight
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
   }
 }
 

@@ -27,6 +27,8 @@ struct StreamW {
   __nv_bfloat16 *qkv, *out, *w13, *w2;
   float *b_qkv, *b_out, *b_w13, *b_w2, *gq, *gk;
   CUtensorMap t_qkv, t_out, t_w13, t_w2;
+  // a bias that is absent or all zero is not added at all
+  bool has_b_qkv = false, has_b_out = false, has_b_w13 = false, has_b_w2 = false;
 };
 struct BlockW {
   StreamW s[2];   // 0 = image stream, 1 = text stream
@@ -45,6 +47,13 @@ struct Bump {
   }
 };
 
+inline bool any_nonzero_bf16(const uint16_t* p, size_t n) {
+  if (!p) return false;
+  for (size_t i = 0; i < n; ++i)
+    if (p[i] & 0x7FFF) return true;
+  return false;
+}
+
 inline float bf16_to_f32(uint16_t b) {
   uint32_t u = uint32_t(b) << 16;
   float f;
@@ -62,6 +71,7 @@ struct lens_dit {
   void* warena = nullptr;
   __nv_bfloat16 *w_t1, *w_t2, *w_txt_in, *w_img_in, *w_proj, *w_mod;
   float *b_t1, *b_t2, *b_txt_in, *b_img_in, *b_proj, *b_mod, *g_txt;
+  bool has_b_txt_in = false, has_b_img_in = false, has_b_proj = false;
   CUtensorMap t_txt_in, t_img_in, t_proj, t_mod;
   std::vector<BlockW> blk;
   // workspace
@@ -281,6 +291,7 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
   }
   if (!(w = L.get("txt_in.weight", {D, kTxtLayers * kTxtDim}, true))) return L.st;
   if ((st = put_bf16(h->w_txt_in, w, (size_t)D * kTxtLayers * kTxtDim))) return st;
+  h->has_b_txt_in = any_nonzero_bf16(L.get("txt_in.bias", {D}, false), D);
   if ((st = put_f32(h->b_txt_in, L.get("txt_in.bias", {D}, false), D, 0.f, stage))) return st;
   // image input, packed [W | W] so the [hi | lo] operand reproduces fp32 tokens
   if (!(w = L.get("img_in.weight", {D, kInCh}, true))) return L.st;
@@ -290,10 +301,12 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
     memcpy(&pack[(size_t)r * 2 * kInCh + kInCh], w + (size_t)r * kInCh, kInCh * 2);
   }
   if ((st = put_bf16(h->w_img_in, pack.data(), pack.size()))) return st;
+  h->has_b_img_in = any_nonzero_bf16(L.get("img_in.bias", {D}, false), D);
   if ((st = put_f32(h->b_img_in, L.get("img_in.bias", {D}, false), D, 0.f, stage))) return st;
   // final layer
   if (!(w = L.get("proj_out.weight", {kInCh, D}, true))) return L.st;
   if ((st = put_bf16(h->w_proj, w, (size_t)kInCh * D))) return st;
+  h->has_b_proj = any_nonzero_bf16(L.get("proj_out.bias", {kInCh}, false), kInCh);
   if ((st = put_f32(h->b_proj, L.get("proj_out.bias", {kInCh}, false), kInCh, 0.f, stage))) return st;
   // all AdaLN projections: block-major, image then text, then norm_out
   const int64_t no_off = (int64_t)nb * kModPerBlock;
@@ -316,6 +329,7 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
       const std::string qkv = p + (s == 0 ? "attn.img_qkv" : "attn.txt_qkv");
       if (!(w = L.get(qkv + ".weight", {3 * D, D}, true))) return L.st;
       if ((st = put_bf16(sw.qkv, w, (size_t)3 * D * D))) return st;
+      sw.has_b_qkv = any_nonzero_bf16(L.get(qkv + ".bias", {3 * D}, false), 3 * D);
       if ((st = put_f32(sw.b_qkv, L.get(qkv + ".bias", {3 * D}, false), 3 * D, 0.f, stage))) return st;
       const std::string nq = p + (s == 0 ? "attn.norm_q" : "attn.norm_added_q");
       const std::string nk = p + (s == 0 ? "attn.norm_k" : "attn.norm_added_k");
@@ -328,6 +342,7 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
       const std::string out = p + (s == 0 ? "attn.to_out" : "attn.to_add_out");
       if (!(w = L.get(out + ".weight", {D, D}, true))) return L.st;
       if ((st = put_bf16(sw.out, w, (size_t)D * D))) return st;
+      sw.has_b_out = any_nonzero_bf16(L.get(out + ".bias", {D}, false), D);
       if ((st = put_f32(sw.b_out, L.get(out + ".bias", {D}, false), D, 0.f, stage))) return st;
 
       const std::string mlp = p + (s == 0 ? "img_mlp" : "txt_mlp");
@@ -346,6 +361,7 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
       const uint16_t* b1 = L.get(mlp + ".w1.bias", {kMlp}, false);
       const uint16_t* b3 = L.get(mlp + ".w3.bias", {kMlp}, false);
       if (L.st) return L.st;
+      sw.has_b_w13 = any_nonzero_bf16(b1, kMlp) || any_nonzero_bf16(b3, kMlp);
       stage.resize(2 * kMlp);
       for (int c = 0; c < kMlp / 32; ++c)
         for (int j = 0; j < 32; ++j) {
@@ -355,6 +371,7 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
       if (cudaMemcpy(sw.b_w13, stage.data(), 2 * kMlp * 4, cudaMemcpyHostToDevice) != cudaSuccess)
         return LENS_ERR_CUDA;
       if ((st = put_bf16(sw.w2, w2, (size_t)D * kMlp))) return st;
+      sw.has_b_w2 = any_nonzero_bf16(L.get(mlp + ".w2.bias", {D}, false), D);
       if ((st = put_f32(sw.b_w2, L.get(mlp + ".w2.bias", {D}, false), D, 0.f, stage))) return st;
     }
   }
@@ -369,10 +386,11 @@ static lens_status make_weight_maps(lens_dit* h) {
             encode_tmap_bf16(&h->t_mod, h->w_mod, h->modw, D, D, 128);
   for (auto& b : h->blk)
     for (auto& s : b.s)
-      ok = ok && encode_tmap_bf16(&s.t_qkv, s.qkv, 3 * D, D, D, kBnQkv) &&
-           encode_tmap_bf16(&s.t_out, s.out, D, D, D, kBnOut) &&
-           encode_tmap_bf16(&s.t_w13, s.w13, 2 * kMlp, D, D, kBnW13) &&
-           encode_tmap_bf16(&s.t_w2, s.w2, D, kMlp, kMlp, kBnW2);
+      // block GEMMs run on CTA pairs: each CTA stages half of the B tile
+      ok = ok && encode_tmap_bf16(&s.t_qkv, s.qkv, 3 * D, D, D, kBnQkv / 2) &&
+           encode_tmap_bf16(&s.t_out, s.out, D, D, D, kBnOut / 2) &&
+           encode_tmap_bf16(&s.t_w13, s.w13, 2 * kMlp, D, D, kBnW13 / 2) &&
+           encode_tmap_bf16(&s.t_w2, s.w2, D, kMlp, kMlp, kBnW2 / 2);
   return ok ? LENS_OK : LENS_ERR_CUDA;
 }
 
@@ -451,7 +469,7 @@ static lens_status text_in_gemm(lens_dit* h, int rows, float* out, cudaStream_t 
   a.p[0] = base_problem(rows, kHidden, kTxtLayers * kTxtDim);
   a.p[0].out_f32 = out;
   a.p[0].ld_out = kHidden;
-  a.p[0].bias = h->b_txt_in;
+  a.p[0].bias = h->has_b_txt_in ? h->b_txt_in : nullptr;
   LENS_LAUNCH(h, 0, st, launch_gemm(kBnTxtIn, EPI_F32, &ta, &h->t_txt_in, nullptr, nullptr, &tc, nullptr, a, h->sms, st));
   return LENS_OK;
 }
@@ -503,7 +521,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
     for (int s = 0; s < np; ++s) {
       const StreamW& w = h->blk[i].s[s];
       GemmProblem p = base_problem(s == 0 ? Mi : Mt, 3 * kHidden, kHidden);
-      p.bias = w.b_qkv;
+      p.bias = w.has_b_qkv ? w.b_qkv : nullptr;
       p.q = h->q;
       p.k = h->k;
       p.v = h->v;
@@ -516,7 +534,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       p.eps = eps;
       a.p[s] = p;
     }
-    LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm(kBnQkv, EPI_QKV, &am.a_img, &wi.t_qkv, np > 1 ? &am.a_txt : nullptr,
+    LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_pair(kBnQkv, EPI_QKV, &am.a_img, &wi.t_qkv, np > 1 ? &am.a_txt : nullptr,
                           np > 1 ? &wt.t_qkv : nullptr, nullptr, nullptr, a, h->sms, st));
   }
   LENS_LAUNCH(h, LENS_KERNEL_ATTENTION, st, launch_joint_attention(h->q, h->k, h->v, B, kHeads, Nt, Ni, h->o_txt, h->o_img, h->err, st));
@@ -528,13 +546,13 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       GemmProblem p = base_problem(s == 0 ? Mi : Mt, kHidden, kHidden);
       p.out_f32 = s == 0 ? hi : ht;
       p.ld_out = kHidden;
-      p.bias = w.b_out;
+      p.bias = w.has_b_out ? w.b_out : nullptr;
       p.gate = (s == 0 ? mI : mT) + 2 * kHidden;
       p.gate_stride = mstride;
       p.rows_per_batch = s == 0 ? Ni : Nt;
       a.p[s] = p;
     }
-    LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm(kBnOut, EPI_RESID, &am.o_img, &wi.t_out, np > 1 ? &am.o_txt : nullptr,
+    LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm_pair(kBnOut, EPI_RESID, &am.o_img, &wi.t_out, np > 1 ? &am.o_txt : nullptr,
                           np > 1 ? &wt.t_out : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
   }
   // MLP branch
@@ -550,10 +568,10 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       const StreamW& w = h->blk[i].s[s];
       GemmProblem p = base_problem(s == 0 ? Mi : Mt, 2 * kMlp, kHidden);
       p.out_bf16 = s == 0 ? h->u_img : h->u_txt;
-      p.bias = w.b_w13;
+      p.bias = w.has_b_w13 ? w.b_w13 : nullptr;
       a.p[s] = p;
     }
-    LENS_LAUNCH(h, LENS_KERNEL_GEMM_W13, st, launch_gemm(kBnW13, EPI_SWIGLU, &am.a_img, &wi.t_w13, np > 1 ? &am.a_txt : nullptr,
+    LENS_LAUNCH(h, LENS_KERNEL_GEMM_W13, st, launch_gemm_pair(kBnW13, EPI_SWIGLU, &am.a_img, &wi.t_w13, np > 1 ? &am.a_txt : nullptr,
                           np > 1 ? &wt.t_w13 : nullptr, &am.uo_img, np > 1 ? &am.uo_txt : nullptr, a, h->sms, st));
   }
   {
@@ -564,13 +582,13 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       GemmProblem p = base_problem(s == 0 ? Mi : Mt, kHidden, kMlp);
       p.out_f32 = s == 0 ? hi : ht;
       p.ld_out = kHidden;
-      p.bias = w.b_w2;
+      p.bias = w.has_b_w2 ? w.b_w2 : nullptr;
       p.gate = (s == 0 ? mI : mT) + 5 * kHidden;
       p.gate_stride = mstride;
       p.rows_per_batch = s == 0 ? Ni : Nt;
       a.p[s] = p;
     }
-    LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm(kBnW2, EPI_RESID, &am.u_img, &wi.t_w2, np > 1 ? &am.u_txt : nullptr,
+    LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm_pair(kBnW2, EPI_RESID, &am.u_img, &wi.t_w2, np > 1 ? &am.u_txt : nullptr,
                           np > 1 ? &wt.t_w2 : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
   }
   return LENS_OK;
@@ -593,7 +611,7 @@ static lens_status run_forward_core(lens_dit* h, int B, int gh, int gw, int Nt, 
     a.p[0] = base_problem(Mi, kHidden, 2 * kInCh);
     a.p[0].out_f32 = h->h_img;
     a.p[0].ld_out = kHidden;
-    a.p[0].bias = h->b_img_in;
+    a.p[0].bias = h->has_b_img_in ? h->b_img_in : nullptr;
     LENS_LAUNCH(h, 0, st, launch_gemm(kBnImgIn, EPI_F32, &tx, &h->t_img_in, nullptr, nullptr, &th, nullptr, a, h->sms, st));
   }
   if (Mt > 0) LENS_CUDA(cudaMemcpyAsync(h->h_txt, h->h_txt0, (size_t)Mt * kHidden * 4, cudaMemcpyDeviceToDevice, st));
@@ -611,7 +629,7 @@ static lens_status run_forward_core(lens_dit* h, int B, int gh, int gw, int Nt, 
     a.p[0] = base_problem(Mi, kInCh, kHidden);
     a.p[0].out_f32 = v_dst;
     a.p[0].ld_out = kInCh;
-    a.p[0].bias = h->b_proj;
+    a.p[0].bias = h->has_b_proj ? h->b_proj : nullptr;
     LENS_LAUNCH(h, 0, st, launch_gemm(kBnProj, EPI_F32, &am.a_img, &h->t_proj, nullptr, nullptr, &tv, nullptr, a, h->sms, st));
   }
   return LENS_OK;
@@ -920,8 +938,9 @@ lens_status lens_op_gemm_bf16(const uint16_t* A, const uint16_t* Bm, const float
   if (!A || !Bm || !C) return LENS_ERR_INVALID_ARG;
   if (M < 1 || N < 32 || K < 64 || K % 64 || N % 32) return LENS_ERR_SHAPE;
   const int bn = N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : (N % 64 == 0 ? 64 : 32));
+  const bool pair = M >= 256 && bn >= 128;     // CTA pairs when a 256-row tile is not mostly padding
   CUtensorMap ta, tb;
-  if (!encode_tmap_bf16(&ta, A, M, K, K, 128) || !encode_tmap_bf16(&tb, Bm, N, K, K, bn))
+  if (!encode_tmap_bf16(&ta, A, M, K, K, 128) || !encode_tmap_bf16(&tb, Bm, N, K, K, pair ? bn / 2 : bn))
     return LENS_ERR_INVALID_ARG;
   CUtensorMap tc;
   if (!encode_tmap_out(&tc, C, 4, M, N, N)) return LENS_ERR_INVALID_ARG;
@@ -933,7 +952,12 @@ lens_status lens_op_gemm_bf16(const uint16_t* A, const uint16_t* Bm, const float
   a.p[0].out_f32 = C;
   a.p[0].ld_out = N;
   a.p[0].bias = bias;
-  LENS_CUDA(launch_gemm(bn, EPI_F32, &ta, &tb, nullptr, nullptr, &tc, nullptr, a, device_sms(), (cudaStream_t)stream));
+  if (pair)
+    LENS_CUDA(launch_gemm_pair(bn, EPI_F32, &ta, &tb, nullptr, nullptr, &tc, nullptr, a, device_sms(),
+                               (cudaStream_t)stream));
+  else
+    LENS_CUDA(launch_gemm(bn, EPI_F32, &ta, &tb, nullptr, nullptr, &tc, nullptr, a, device_sms(),
+                          (cudaStream_t)stream));
   return LENS_OK;
 }
 
