@@ -29,22 +29,23 @@ __device__ __forceinline__ float ex2(float x) {
 //               exponentials run, and the two tiles ping-pong on the tensor cores
 //   warp 8      TMA: both Q tiles once, then K and V tiles of 128 keys (3 stages)
 //   warp 9      UMMA issuer: S_X = Q_X K_j^T (M=128, N=128, K=64) and
-//               O_X += P_X V_j (M=128, N=64, K=128)
+//               O_X += P_X V_j (M=128, N=64, K=128) with P_X read from TMEM
 // The running max m and sum l of each row live in registers; O_X is rescaled in
 // TMEM only when m grows by more than 2^8 (softmax is invariant to the subtracted
 // constant, so a stale max is exact up to rounding).
-// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,320), O_1 [320,384).
+// P_X goes from the softmax registers into TMEM (two bf16 per column) and is the A
+// operand of P V there, so neither P nor its operand reads touch shared memory.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,320), O_1 [320,384),
+// P_0 [384,448), P_1 [448,512).
 namespace tc {
 
 constexpr int BQ = 128, BKV = 128, STAGES = 3, TILES = 2;
 constexpr int THREADS = 320;
 constexpr uint32_t Q_BYTES = BQ * 64 * 2;          // 16 KB per query tile
 constexpr uint32_t KV_BYTES = BKV * 64 * 2;        // 16 KB each for K and V
-constexpr uint32_t P_BYTES = BQ * BKV * 2;         // 32 KB per query tile: two 64-key swizzle atoms
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_KV = OFF_Q + TILES * Q_BYTES;
-constexpr uint32_t OFF_P = OFF_KV + STAGES * 2 * KV_BYTES;
-constexpr uint32_t OFF_BAR = OFF_P + TILES * P_BYTES;
+constexpr uint32_t OFF_BAR = OFF_KV + STAGES * 2 * KV_BYTES;
 constexpr size_t SMEM = 1024 + OFF_BAR + 256;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
@@ -68,7 +69,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = sm + OFF_Q;
   uint8_t* sKV = sm + OFF_KV;
-  uint8_t* sP = sm + OFF_P;
   Bars& bar = *reinterpret_cast<Bars*>(sm + OFF_BAR);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -169,12 +169,11 @@ __global__ void __launch_bounds__(THREADS, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t pbase = smem_u32(sP + x * P_BYTES);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint64_t pdesc = umma_desc_sw128(pbase + (k >> 2) * (BQ * 128) + (k & 3) * 32);
+            for (int k = 0; k < 8; ++k) {              // 16 keys = 8 TMEM columns of P per step
               const uint64_t vdesc = umma_desc_sw128_mn(vbase + k * 2048);
-              umma_bf16(tmem + 256 + x * 64, pdesc, vdesc, idesc_pv, (jj > 0 || k > 0) ? 1u : 0u);
+              umma_bf16_ts(tmem + 256 + x * 64, tmem + 384 + x * 64 + 8 * k, vdesc, idesc_pv,
+                           (jj > 0 || k > 0) ? 1u : 0u);
             }
             umma_commit(&bar.pv_done[x]);
           }
@@ -190,8 +189,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;           // TMEM lane quarter
     const int r = quarter * 32 + lane;      // row inside the tile
     const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
-    const uint32_t s_col = x * 128, o_col = 256 + x * 64;
-    uint8_t* Px = sP + x * P_BYTES;
+    const uint32_t s_col = x * 128, o_col = 256 + x * 64, p_col = 384 + x * 64;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
@@ -244,29 +242,22 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, corr != 1.f)) {
+      }
+      // P row r -> TMEM, column c = keys (2c, 2c + 1)
+      tmem_st32_u(lane_addr + p_col, pk);
+      tmem_st32_u(lane_addr + p_col + 32, pk + 32);
+      if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            float o[32];
-            tmem_ld32(lane_addr + o_col + c * 32, o);
-            tmem_ld_wait();
+        for (int c = 0; c < 2; ++c) {
+          float o[32];
+          tmem_ld32(lane_addr + o_col + c * 32, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= corr;
-            tmem_st32(lane_addr + o_col + c * 32, o);
-          }
-          tmem_st_wait();
+          for (int i = 0; i < 32; ++i) o[i] *= corr;
+          tmem_st32(lane_addr + o_col + c * 32, o);
         }
       }
-      // P row r -> two 64-key atoms, 128-byte swizzle (16-byte chunk c of the row
-      // goes to position c ^ (r & 7))
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint32_t addr = smem_u32(Px) + (c >> 3) * (BQ * 128) + r * 128 + ((((c & 7) ^ (r & 7))) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * c]), "r"(pk[4 * c + 1]),
-                     "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
-                     : "memory");
-      }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.p_full[x]);
