@@ -70,9 +70,8 @@ def kernel_work(kernel: str, B: int, n_img: int, n_txt: int):
         return "flop", 2.0 * M * D * 2 * F
     if kernel == "gemm_w2":
         return "flop", 2.0 * M * F * D
-    if kernel == "rmsnorm_mod":   # one stream per launch; average over image and text launches
-        rows = B * (n_img + n_txt) / 2.0
-        return "byte", rows * D * (4 + 2)
+    if kernel == "rmsnorm_mod":   # both streams in one launch: fp32 row in, bf16 row out
+        return "byte", B * (n_img + n_txt) * D * (4.0 + 2.0)
     if kernel == "gemm_mod":
         return "byte", (48 * 2 * 9216 + 3072) * D * 2.0
     raise ValueError(kernel)
@@ -105,6 +104,55 @@ def dram_traffic(kernel: str, workload: str):
                 rec.get("source_hash") == source_hash(kernel):
             return rec.get("dram_bytes_per_launch")
     return None
+
+
+# ---------------------------------------------------------------- replica plumbing
+class EventTimer:
+    """Device timing with CUDA events on the launching stream."""
+
+    def __init__(self, stream):
+        import torch
+        self.stream = stream
+        self.ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    def start(self):
+        self.ev[0].record(self.stream)
+
+    def stop(self):
+        self.ev[1].record(self.stream)
+
+    def elapsed_ms(self) -> float:
+        return self.ev[0].elapsed_time(self.ev[1])
+
+
+def timed_region(step, steps: int, barrier, sync, timer) -> float:
+    """Barrier + synchronize, time exactly `steps` calls of step(), synchronize +
+    barrier; returns this rank's elapsed milliseconds."""
+    barrier()
+    sync()
+    timer.start()
+    for _ in range(steps):
+        step()
+    timer.stop()
+    sync()
+    barrier()
+    return timer.elapsed_ms()
+
+
+def max_over_ranks(values, dist, device) -> list:
+    """Element-wise max of per-rank values (identity without a process group)."""
+    if dist is None:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_value(units_per_step_per_rank: float, n_ranks: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the units every rank processed per step / the slowest
+    rank's time per step (weak scaling: each rank runs its own replica)."""
+    return n_ranks * units_per_step_per_rank / (ms_per_step / 1e3)
 
 
 # ---------------------------------------------------------------- clocks
@@ -221,6 +269,13 @@ def main():
     import flow_matching_mmdit_b200 as L
 
     torch.cuda.set_device(local)
+    # a created stream: the library captures each sampler call as a CUDA graph there
+    work_stream = torch.cuda.Stream()
+    with torch.cuda.stream(work_stream):
+        return _run_lens(args, wl, config, world, rank, local, torch, L)
+
+
+def _run_lens(args, wl, config, world, rank, local, torch, L):
     dist = None
     if world > 1:
         import datetime
@@ -260,20 +315,10 @@ def main():
     # ------------------------------------------------ timed region (device-resident inputs)
     uuid = str(torch.cuda.get_device_properties(local).uuid)
     launches0 = L.lens_dit_launch_count(h)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier = dist.barrier if dist else (lambda: None)
     with ClockSampler(uuid) as clk:
-        if dist:
-            dist.barrier()
-        torch.cuda.synchronize()
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        if dist:
-            dist.barrier()
+        ms_total = timed_region(step, args.steps, barrier, torch.cuda.synchronize, EventTimer(stream))
     L.lens_dit_sync(h)
-    ms_total = ev0.elapsed_time(ev1)
     gpu_launches = L.lens_dit_launch_count(h) - launches0
     k_launches, k_ms = L.lens_dit_profile_read(h)
     L.lens_dit_profile_kernel(h, "none", 0)
@@ -288,33 +333,21 @@ def main():
                             seed, out)
         out_pinned.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.steps):
+    def e2e_step():
         txt_dev.copy_(txt_pinned, non_blocking=True)
         L.lens_sample_euler(h, txt_dev, None, wl.batch, wl.n_txt, wl.height_px, wl.width_px, wl.steps, wl.guidance,
                             seed, out)
         out_pinned.copy_(out, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    L.lens_dit_sync(h)
-    e2e_ms = e0.elapsed_time(e1)
-    assert np.all(np.isfinite(out_pinned.numpy()))
 
-    if dist:
-        t = torch.tensor([ms_total, e2e_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, e2e_ms = float(t[0]), float(t[1])
+    e2e_ms = timed_region(e2e_step, args.steps, barrier, torch.cuda.synchronize, EventTimer(stream))
+    L.lens_dit_sync(h)
+    assert np.all(np.isfinite(out_pinned.numpy()))
+    ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], dist, "cuda")
 
     ms_step = ms_total / args.steps
     tokens_per_step = wl.batch * wl.n_img * wl.steps
-    value = args.gpus * tokens_per_step / (ms_step / 1e3)
-    e2e_value = args.gpus * tokens_per_step / (e2e_ms / args.steps / 1e3)
+    value = job_value(tokens_per_step, args.gpus, ms_step)
+    e2e_value = job_value(tokens_per_step, args.gpus, e2e_ms / args.steps)
     flops_step = wl.steps * config["forward_rows"] * forward_flops(wl.n_img, wl.n_txt)
     peaks = measured_peaks()
     tflops = flops_step / (ms_step / 1e3) / 1e12

@@ -80,11 +80,26 @@ struct lens_dit {
   float *h_img, *h_txt, *h_txt0, *vtok, *xtok, *tfeat, *hid, *temb, *mod;
   float2* rope;
   int* err;
+  // the last sampler call, captured as a CUDA graph and replayed for identical calls
+  struct SampleGraph {
+    bool valid = false;
+    const void *txt_cond, *txt_uncond, *latent_out;
+    cudaStream_t stream;
+    int B, n_txt, height_px, width_px, steps;
+    float guidance;
+    uint64_t seed;
+    int prof_kind;
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    int64_t launches = 0;        // kernels one replay runs
+  } sg;
   // measurement
   int64_t launches = 0;
   int prof_kind = 0, prof_cap = 0, prof_n = 0;
   std::vector<cudaEvent_t> prof_ev;
 };
+
+static void drop_sample_graph(lens_dit* h);
 
 // ============================================================ helpers
 static const char* kStatusStr[] = {"ok", "invalid argument", "shape out of range", "out of device memory",
@@ -652,6 +667,42 @@ static lens_status check_model_fields(const lens_dit_config* c) {
   return LENS_OK;
 }
 
+static void drop_sample_graph(lens_dit* h) {
+  if (h->sg.exec) cudaGraphExecDestroy(h->sg.exec);
+  if (h->sg.graph) cudaGraphDestroy(h->sg.graph);
+  h->sg = lens_dit::SampleGraph();
+}
+
+// Enqueue one sampler call on `st` (validated arguments).
+static lens_status enqueue_sample(lens_dit* h, const uint16_t* txt_cond, const uint16_t* txt_uncond, int B,
+                                  int n_txt, int gh, int gw, int steps, float guidance, uint64_t seed,
+                                  float* latent_out, cudaStream_t st) {
+  const bool cfg = guidance != 1.0f;
+  const int Ni = gh * gw;
+  const int Bf = cfg ? 2 * B : B;
+  const int64_t per_sample = (int64_t)Ni * kInCh;
+  lens_status s;
+  LENS_LAUNCH(h, 0, st, launch_noise_tokens(seed, B, gh, gw, h->xtok, st));
+  LENS_LAUNCH(h, 0, st, launch_tokens_to_operand(h->xtok, (int64_t)B * Ni, cfg ? 2 : 1, (int64_t)B * Ni, h->xin, st));
+  if ((s = text_norm_rows(h, txt_cond, B * n_txt, 0, st))) return s;
+  if (cfg && (s = text_norm_rows(h, txt_uncond, B * n_txt, B * n_txt, st))) return s;
+  if ((s = text_in_gemm(h, Bf * n_txt, h->h_txt0, st))) return s;
+
+  const int chunk = h->cfg.max_timesteps;
+  float tv[kMaxTimesteps];
+  for (int k0 = 0; k0 < steps; k0 += chunk) {
+    const int T = steps - k0 < chunk ? steps - k0 : chunk;
+    for (int j = 0; j < T; ++j) tv[j] = (float)(1.0 - (double)(k0 + j) / (double)steps);
+    if ((s = compute_modulation(h, tv, T, st))) return s;
+    for (int j = 0; j < T; ++j) {
+      if ((s = run_forward_core(h, Bf, gh, gw, n_txt, h->mod + (int64_t)j * h->modw, 0, h->vtok, st))) return s;
+      LENS_LAUNCH(h, 0, st, launch_euler_cfg(h->xtok, h->vtok, per_sample, B, cfg, 1.0f / (float)steps, guidance, h->xin, st));
+    }
+  }
+  LENS_LAUNCH(h, 0, st, launch_unpatchify(h->xtok, B, gh, gw, latent_out, st));
+  return LENS_OK;
+}
+
 // ============================================================ C ABI
 extern "C" {
 
@@ -740,6 +791,7 @@ lens_status lens_dit_create(const lens_dit_config* cfg, const lens_weight* w, in
 void lens_dit_destroy(lens_dit* h) {
   if (!h) return;
   cudaDeviceSynchronize();
+  drop_sample_graph(h);
   for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
   if (h->ws) cudaFree(h->ws);
   if (h->warena) cudaFree(h->warena);
@@ -809,32 +861,57 @@ lens_status lens_sample_euler(lens_dit* h, const uint16_t* txt_cond, const uint1
   if (steps < 1 || !isfinite(guidance)) return LENS_ERR_INVALID_ARG;
   if (height_px <= 0 || width_px <= 0 || height_px % 16 || width_px % 16) return LENS_ERR_SHAPE;
   const bool cfg = guidance != 1.0f;
-  const int gh = height_px / 16, gw = width_px / 16, Ni = gh * gw;
+  const int gh = height_px / 16, gw = width_px / 16;
   const int Bf = cfg ? 2 * B : B;
   lens_status s = check_sizes(h, Bf, gh, gw, n_txt);
   if (s) return s;
   if (B < 1) return LENS_ERR_SHAPE;
   cudaStream_t st = (cudaStream_t)stream;
-  const int64_t per_sample = (int64_t)Ni * kInCh;
-
-  LENS_LAUNCH(h, 0, st, launch_noise_tokens(seed, B, gh, gw, h->xtok, st));
-  LENS_LAUNCH(h, 0, st, launch_tokens_to_operand(h->xtok, (int64_t)B * Ni, cfg ? 2 : 1, (int64_t)B * Ni, h->xin, st));
-  if ((s = text_norm_rows(h, txt_cond, B * n_txt, 0, st))) return s;
-  if (cfg && (s = text_norm_rows(h, txt_uncond, B * n_txt, B * n_txt, st))) return s;
-  if ((s = text_in_gemm(h, Bf * n_txt, h->h_txt0, st))) return s;
-
-  const int chunk = h->cfg.max_timesteps;
-  float tv[kMaxTimesteps];
-  for (int k0 = 0; k0 < steps; k0 += chunk) {
-    const int T = steps - k0 < chunk ? steps - k0 : chunk;
-    for (int j = 0; j < T; ++j) tv[j] = (float)(1.0 - (double)(k0 + j) / (double)steps);
-    if ((s = compute_modulation(h, tv, T, st))) return s;
-    for (int j = 0; j < T; ++j) {
-      if ((s = run_forward_core(h, Bf, gh, gw, n_txt, h->mod + (int64_t)j * h->modw, 0, h->vtok, st))) return s;
-      LENS_LAUNCH(h, 0, st, launch_euler_cfg(h->xtok, h->vtok, per_sample, B, cfg, 1.0f / (float)steps, guidance, h->xin, st));
-    }
+  if (!cfg) txt_uncond = nullptr;
+  // On a created stream the call is captured once as a CUDA graph and replayed
+  // while the arguments stay the same (the legacy default stream cannot capture).
+  if (st == nullptr) return enqueue_sample(h, txt_cond, txt_uncond, B, n_txt, gh, gw, steps, guidance, seed, latent_out, st);
+  lens_dit::SampleGraph& g = h->sg;
+  if (g.valid && g.txt_cond == txt_cond && g.txt_uncond == txt_uncond && g.latent_out == latent_out &&
+      g.stream == st && g.B == B && g.n_txt == n_txt && g.height_px == height_px && g.width_px == width_px &&
+      g.steps == steps && g.guidance == guidance && g.seed == seed && g.prof_kind == h->prof_kind) {
+    LENS_CUDA(cudaGraphLaunch(g.exec, st));
+    h->launches += g.launches;
+    return LENS_OK;
   }
-  LENS_LAUNCH(h, 0, st, launch_unpatchify(h->xtok, B, gh, gw, latent_out, st));
+  drop_sample_graph(h);
+  const int64_t l0 = h->launches;
+  if (cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return LENS_ERR_CUDA;
+  s = enqueue_sample(h, txt_cond, txt_uncond, B, n_txt, gh, gw, steps, guidance, seed, latent_out, st);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t ce = cudaStreamEndCapture(st, &graph);
+  if (s != LENS_OK || ce != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    cudaGetLastError();
+    return s != LENS_OK ? s : LENS_ERR_CUDA;
+  }
+  cudaGraphExec_t exec = nullptr;
+  if (cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
+    cudaGraphDestroy(graph);
+    return LENS_ERR_CUDA;
+  }
+  g.valid = true;
+  g.txt_cond = txt_cond;
+  g.txt_uncond = txt_uncond;
+  g.latent_out = latent_out;
+  g.stream = st;
+  g.B = B;
+  g.n_txt = n_txt;
+  g.height_px = height_px;
+  g.width_px = width_px;
+  g.steps = steps;
+  g.guidance = guidance;
+  g.seed = seed;
+  g.prof_kind = h->prof_kind;
+  g.graph = graph;
+  g.exec = exec;
+  g.launches = h->launches - l0;
+  LENS_CUDA(cudaGraphLaunch(exec, st));
   return LENS_OK;
 }
 
@@ -842,6 +919,7 @@ lens_status lens_dit_profile_kernel(lens_dit* h, lens_kernel kernel, int capacit
   if (!h || capacity < 0) return LENS_ERR_INVALID_ARG;
   if ((int)kernel < 0 || (int)kernel > 7) return LENS_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return LENS_ERR_CUDA;
+  drop_sample_graph(h);                 // a captured graph may record the old events
   for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
   h->prof_ev.clear();
   h->prof_kind = 0;
