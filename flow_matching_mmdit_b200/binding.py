@@ -25,7 +25,8 @@ EXPORTS = [
     "lens_op_unpatchify", "lens_op_rope_table", "lens_op_rmsnorm_modulate", "lens_op_gemm_bf16",
     "lens_op_attention", "lens_op_euler_cfg", "lens_dit_op_timestep", "lens_dit_op_text_input",
     "lens_device_sm_count", "lens_dit_profile_kernel", "lens_dit_profile_read", "lens_dit_launch_count",
-    "lens_op_timestep_embed_noalloc",
+    "lens_op_timestep_embed_noalloc", "lens_dit_forward_masked", "lens_sample_euler_masked",
+    "lens_op_attention_masked",
 ]
 
 KERNELS = {"none": 0, "attention": 1, "gemm_qkv": 2, "gemm_out": 3, "gemm_w13": 4, "gemm_w2": 5, "rmsnorm_mod": 6,
@@ -89,6 +90,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lens_dit_profile_read": (I, [P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]),
         "lens_dit_launch_count": (L, [P]),
         "lens_op_timestep_embed_noalloc": (I, [P, I, P, P, P, P, P, P]),
+        "lens_dit_forward_masked": (I, [P, P, I, I, I, P, I, P, P, P, P]),
+        "lens_sample_euler_masked": (I, [P, P, P, P, P, I, I, I, I, I, F, U64, P, P]),
+        "lens_op_attention_masked": (I, [P, P, P, I, I, I, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -178,6 +182,32 @@ def lens_dit_forward(h: LensDit, img_tokens, B: int, grid_h: int, grid_w: int, t
                                            tt.ctypes.data, _ptr(v_out), _stream(stream)), "lens_dit_forward")
 
 
+def _ints(a) -> Optional[np.ndarray]:
+    return None if a is None else np.ascontiguousarray(np.asarray(a, np.int32))
+
+
+def _iptr(a) -> Optional[int]:
+    return None if a is None else a.ctypes.data
+
+
+def lens_dit_forward_masked(h: LensDit, img_tokens, B: int, grid_h: int, grid_w: int, txt, n_txt: int,
+                            txt_len: Optional[Sequence[int]], t: Sequence[float], v_out, stream=None) -> None:
+    tt = np.ascontiguousarray(np.asarray(t, np.float32))
+    ln = _ints(txt_len)
+    _check(load_library().lens_dit_forward_masked(h.ptr, _ptr(img_tokens), B, grid_h, grid_w, _ptr(txt), n_txt,
+                                                  _iptr(ln), tt.ctypes.data, _ptr(v_out), _stream(stream)),
+           "lens_dit_forward_masked")
+
+
+def lens_sample_euler_masked(h: LensDit, txt_cond, len_cond, txt_uncond, len_uncond, B: int, n_txt: int,
+                             height_px: int, width_px: int, steps: int, guidance: float, seed: int, latent_out,
+                             stream=None) -> None:
+    lc, lu = _ints(len_cond), _ints(len_uncond)
+    _check(load_library().lens_sample_euler_masked(h.ptr, _ptr(txt_cond), _iptr(lc), _ptr(txt_uncond), _iptr(lu), B,
+                                                   n_txt, height_px, width_px, steps, guidance, seed,
+                                                   _ptr(latent_out), _stream(stream)), "lens_sample_euler_masked")
+
+
 def lens_sample_euler(h: LensDit, txt_cond, txt_uncond, B: int, n_txt: int, height_px: int, width_px: int,
                       steps: int, guidance: float, seed: int, latent_out, stream=None) -> None:
     _check(load_library().lens_sample_euler(h.ptr, _ptr(txt_cond), _ptr(txt_uncond), B, n_txt, height_px, width_px,
@@ -246,6 +276,14 @@ def lens_op_gemm_bf16(A, Bm, bias, C, M: int, N: int, K: int, stream=None) -> No
 def lens_op_attention(q, k, v, B: int, n_txt: int, n_img: int, out_txt, out_img, stream=None) -> None:
     _check(load_library().lens_op_attention(_ptr(q), _ptr(k), _ptr(v), B, n_txt, n_img, _ptr(out_txt),
                                             _ptr(out_img), _stream(stream)), "lens_op_attention")
+
+
+def lens_op_attention_masked(q, k, v, B: int, n_txt: int, n_img: int, txt_len, out_txt, out_img,
+                             stream=None) -> None:
+    ln = _ints(txt_len)
+    _check(load_library().lens_op_attention_masked(_ptr(q), _ptr(k), _ptr(v), B, n_txt, n_img, _iptr(ln),
+                                                   _ptr(out_txt), _ptr(out_img), _stream(stream)),
+           "lens_op_attention_masked")
 
 
 def lens_op_euler_cfg(x, v_cond, v_uncond, n: int, dt: float, guidance: float, stream=None) -> None:

@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     joint_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                               const __grid_constant__ CUtensorMap tmV, int N, int n_txt, int heads,
                               __nv_bfloat16* __restrict__ out_txt, __nv_bfloat16* __restrict__ out_img,
-                              float scale_log2, int* err) {
+                              float scale_log2, const TextLengths txt_len, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = sm + OFF_Q;
@@ -76,6 +76,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int bh = b * heads + h;
   const int q0 = blockIdx.x * (TILES * BQ);
   const int nkv = (N + BKV - 1) / BKV;
+  // text keys [txt_valid, n_txt) of this batch row are padding and never attended
+  const int txt_valid = txt_len.n[b] < n_txt ? txt_len.n[b] : n_txt;
+  const int txt_pad_end = n_txt;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar.q_full, 1);
@@ -211,6 +214,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < 128; ++i)
           if (j * BKV + i >= N) sc[i] = -INFINITY;
       }
+      if (j * BKV < txt_pad_end && (j + 1) * BKV > txt_valid) {   // padded text keys of this sample
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (j * BKV + i >= txt_valid && j * BKV + i < txt_pad_end) sc[i] = -INFINITY;
+      }
       // 8 independent partial maxima / sums keep the dependency chains short
       float pm[8];
 #pragma unroll
@@ -224,12 +232,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         corr = ex2(m - mx);
         m = mx;
       }
+      // every key seen so far masked: m is still -inf and so is every score here
+      const float m_base = m == -INFINITY ? 0.f : m;
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       uint32_t pk[64];
 #pragma unroll
       for (int i = 0; i < 128; i += 2) {
-        const float e0 = ex2(fmaf(sc[i], scale_log2, -m));
-        const float e1 = ex2(fmaf(sc[i + 1], scale_log2, -m));
+        const float e0 = ex2(fmaf(sc[i], scale_log2, -m_base));
+        const float e1 = ex2(fmaf(sc[i + 1], scale_log2, -m_base));
         ps[i & 7] += e0;
         ps[(i + 1) & 7] += e1;
         pk[i >> 1] = pack_bf16x2(e0, e1);
@@ -304,9 +314,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 cudaError_t launch_joint_attention(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int B,
                                    int heads, int n_txt, int n_img, __nv_bfloat16* out_txt, __nv_bfloat16* out_img,
-                                   int* err, cudaStream_t st) {
+                                   const TextLengths* txt_len, int* err, cudaStream_t st) {
   const int N = n_txt + n_img;
   if (N <= 0 || B <= 0) return cudaSuccess;
+  if (B > kMaxRows) return cudaErrorInvalidValue;
+  TextLengths lens;
+  for (int b = 0; b < kMaxRows; ++b) lens.n[b] = (txt_len && b < B) ? txt_len->n[b] : n_txt;
   // [B*heads, N, 64] views: tiles of 128 rows never cross into the next head, and
   // rows past N read as zeros
   CUtensorMap tq, tk, tv;
@@ -324,7 +337,7 @@ cudaError_t launch_joint_attention(const __nv_bfloat16* q, const __nv_bfloat16* 
   dim3 grid((N + tc::TILES * tc::BQ - 1) / (tc::TILES * tc::BQ), heads, B);
   const float scale_log2 = 0.125f * 1.4426950408889634f;
   tc::joint_attention_tc_kernel<<<grid, tc::THREADS, tc::SMEM, st>>>(tq, tk, tv, N, n_txt, heads, out_txt, out_img,
-                                                            scale_log2, err);
+                                                                        scale_log2, lens, err);
   return cudaGetLastError();
 }
 

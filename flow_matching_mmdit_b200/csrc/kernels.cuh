@@ -27,10 +27,16 @@ struct TimestepList {
   int T;
 };
 
-// attention.cu
+// Valid text lengths per batch row (text keys at and past n[b] are padding).
+constexpr int kMaxRows = 64;
+struct TextLengths {
+  int n[kMaxRows];
+};
+
+// attention.cu (txt_len == nullptr: every text key is valid)
 cudaError_t launch_joint_attention(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int B,
                                    int heads, int n_txt, int n_img, __nv_bfloat16* out_txt, __nv_bfloat16* out_img,
-                                   int* err, cudaStream_t st);
+                                   const TextLengths* txt_len, int* err, cudaStream_t st);
 
 // elementwise.cu
 cudaError_t launch_noise_tokens(uint64_t seed, int B, int gh, int gw, float* tokens, cudaStream_t st);

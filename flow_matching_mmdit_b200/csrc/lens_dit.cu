@@ -89,6 +89,8 @@ struct lens_dit {
     float guidance;
     uint64_t seed;
     int prof_kind;
+    bool masked;
+    TextLengths lens;
     cudaGraph_t graph = nullptr;
     cudaGraphExec_t exec = nullptr;
     int64_t launches = 0;        // kernels one replay runs
@@ -119,11 +121,13 @@ struct KScope {
   KScope(lens_dit* h_, int kind, cudaStream_t st_) : h(h_), st(st_), on(false) {
     ++h->launches;
     if (h->prof_kind == kind && h->prof_n < h->prof_cap) {
-      on = cudaEventRecord(h->prof_ev[2 * h->prof_n], st) == cudaSuccess;
+      // external records become real event nodes when the stream is being captured
+      on = cudaEventRecordWithFlags(h->prof_ev[2 * h->prof_n], st, cudaEventRecordExternal) == cudaSuccess;
     }
   }
   ~KScope() {
-    if (on && cudaEventRecord(h->prof_ev[2 * h->prof_n + 1], st) == cudaSuccess) ++h->prof_n;
+    if (on && cudaEventRecordWithFlags(h->prof_ev[2 * h->prof_n + 1], st, cudaEventRecordExternal) == cudaSuccess)
+      ++h->prof_n;
   }
 };
 
@@ -515,7 +519,7 @@ static lens_status make_act_maps(lens_dit* h, int Mi, int Mt, float* hi, float* 
 
 // One dual-stream block on residual streams hi [B*Ni, 1536], ht [B*Nt, 1536].
 static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, int Ni, int Nt, const float* mod,
-                             int64_t mstride, const ActMaps& am, cudaStream_t st) {
+                             int64_t mstride, const ActMaps& am, const TextLengths* tl, cudaStream_t st) {
   const float eps = h->cfg.eps;
   const int Mi = B * Ni, Mt = B * Nt, N = Ni + Nt;
   const float* mI = mod + (int64_t)i * kModPerBlock;
@@ -552,7 +556,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
     LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_pair(kBnQkv, EPI_QKV, &am.a_img, &wi.t_qkv, np > 1 ? &am.a_txt : nullptr,
                           np > 1 ? &wt.t_qkv : nullptr, nullptr, nullptr, a, h->sms, st));
   }
-  LENS_LAUNCH(h, LENS_KERNEL_ATTENTION, st, launch_joint_attention(h->q, h->k, h->v, B, kHeads, Nt, Ni, h->o_txt, h->o_img, h->err, st));
+  LENS_LAUNCH(h, LENS_KERNEL_ATTENTION, st, launch_joint_attention(h->q, h->k, h->v, B, kHeads, Nt, Ni, h->o_txt, h->o_img, tl, h->err, st));
   {
     GemmArgs a = make_args(h->err);
     a.num_problems = np;
@@ -612,7 +616,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
 // Whole forward: h->xin holds the [hi | lo] token operand [B*Ni, 256] and h->h_txt0
 // the text input [B*Nt, 1536]; velocity tokens go to v_dst [B*Ni, 128].
 static lens_status run_forward_core(lens_dit* h, int B, int gh, int gw, int Nt, const float* mod, int64_t mstride,
-                                    float* v_dst, cudaStream_t st) {
+                                    float* v_dst, const TextLengths* tl, cudaStream_t st) {
   const int Ni = gh * gw, Mi = B * Ni, Mt = B * Nt;
   lens_status s;
   LENS_LAUNCH(h, 0, st, launch_rope_table(gh, gw, Nt, h->rope, st));
@@ -633,7 +637,7 @@ static lens_status run_forward_core(lens_dit* h, int B, int gh, int gw, int Nt, 
   ActMaps am;
   if ((s = make_act_maps(h, Mi, Mt, h->h_img, h->h_txt, am))) return s;
   for (int i = 0; i < h->cfg.num_blocks; ++i)
-    if ((s = run_block(h, i, h->h_img, h->h_txt, B, Ni, Nt, mod, mstride, am, st))) return s;
+    if ((s = run_block(h, i, h->h_img, h->h_txt, B, Ni, Nt, mod, mstride, am, tl, st))) return s;
   const float* no = mod + (int64_t)h->cfg.num_blocks * kModPerBlock;   // (scale, shift)
   LENS_LAUNCH(h, LENS_KERNEL_RMSNORM_MOD, st, launch_rmsnorm_modulate(h->h_img, Mi, Ni, no + kHidden, no, mstride, h->cfg.eps, h->a_img, st));
   {
@@ -676,7 +680,7 @@ static void drop_sample_graph(lens_dit* h) {
 // Enqueue one sampler call on `st` (validated arguments).
 static lens_status enqueue_sample(lens_dit* h, const uint16_t* txt_cond, const uint16_t* txt_uncond, int B,
                                   int n_txt, int gh, int gw, int steps, float guidance, uint64_t seed,
-                                  float* latent_out, cudaStream_t st) {
+                                  float* latent_out, const TextLengths* tl, cudaStream_t st) {
   const bool cfg = guidance != 1.0f;
   const int Ni = gh * gw;
   const int Bf = cfg ? 2 * B : B;
@@ -695,7 +699,7 @@ static lens_status enqueue_sample(lens_dit* h, const uint16_t* txt_cond, const u
     for (int j = 0; j < T; ++j) tv[j] = (float)(1.0 - (double)(k0 + j) / (double)steps);
     if ((s = compute_modulation(h, tv, T, st))) return s;
     for (int j = 0; j < T; ++j) {
-      if ((s = run_forward_core(h, Bf, gh, gw, n_txt, h->mod + (int64_t)j * h->modw, 0, h->vtok, st))) return s;
+      if ((s = run_forward_core(h, Bf, gh, gw, n_txt, h->mod + (int64_t)j * h->modw, 0, h->vtok, tl, st))) return s;
       LENS_LAUNCH(h, 0, st, launch_euler_cfg(h->xtok, h->vtok, per_sample, B, cfg, 1.0f / (float)steps, guidance, h->xin, st));
     }
   }
@@ -820,7 +824,21 @@ static lens_status check_sizes(lens_dit* h, int B, int gh, int gw, int n_txt) {
 
 lens_status lens_dit_forward(lens_dit* h, const float* img_tokens, int B, int grid_h, int grid_w,
                              const uint16_t* txt, int n_txt, const float* t, float* v_out, void* stream) {
+  return lens_dit_forward_masked(h, img_tokens, B, grid_h, grid_w, txt, n_txt, nullptr, t, v_out, stream);
+}
+
+lens_status lens_dit_forward_masked(lens_dit* h, const float* img_tokens, int B, int grid_h, int grid_w,
+                                    const uint16_t* txt, int n_txt, const int* txt_len, const float* t, float* v_out,
+                                    void* stream) {
   if (!h || !img_tokens || !t || !v_out || (n_txt > 0 && !txt)) return LENS_ERR_INVALID_ARG;
+  TextLengths tl;
+  if (txt_len) {
+    if (B > kMaxRows) return LENS_ERR_SHAPE;
+    for (int b = 0; b < B; ++b) {
+      if (txt_len[b] < 0 || txt_len[b] > n_txt) return LENS_ERR_SHAPE;
+      tl.n[b] = txt_len[b];
+    }
+  }
   lens_status s = check_sizes(h, B, grid_h, grid_w, n_txt);
   if (s) return s;
   if (B > h->cfg.max_timesteps) return LENS_ERR_SHAPE;
@@ -832,7 +850,7 @@ lens_status lens_dit_forward(lens_dit* h, const float* img_tokens, int B, int gr
   LENS_LAUNCH(h, 0, st, launch_tokens_to_operand(img_tokens, (int64_t)B * Ni, 1, 0, h->xin, st));
   if ((s = text_norm_rows(h, txt, B * n_txt, 0, st))) return s;
   if ((s = text_in_gemm(h, B * n_txt, h->h_txt0, st))) return s;
-  return run_forward_core(h, B, grid_h, grid_w, n_txt, h->mod, h->modw, v_out, st);
+  return run_forward_core(h, B, grid_h, grid_w, n_txt, h->mod, h->modw, v_out, txt_len ? &tl : nullptr, st);
 }
 
 lens_status lens_dit_debug_blocks(lens_dit* h, int first, int last, float* h_img, float* h_txt, int B, int grid_h,
@@ -850,13 +868,21 @@ lens_status lens_dit_debug_blocks(lens_dit* h, int first, int last, float* h_img
   ActMaps am;
   if ((s = make_act_maps(h, B * Ni, B * n_txt, h_img, h_txt, am))) return s;
   for (int i = first; i < last; ++i)
-    if ((s = run_block(h, i, h_img, h_txt, B, Ni, n_txt, h->mod, h->modw, am, st))) return s;
+    if ((s = run_block(h, i, h_img, h_txt, B, Ni, n_txt, h->mod, h->modw, am, nullptr, st))) return s;
   return LENS_OK;
 }
 
 lens_status lens_sample_euler(lens_dit* h, const uint16_t* txt_cond, const uint16_t* txt_uncond, int B, int n_txt,
                               int height_px, int width_px, int steps, float guidance, uint64_t seed,
                               float* latent_out, void* stream) {
+  return lens_sample_euler_masked(h, txt_cond, nullptr, txt_uncond, nullptr, B, n_txt, height_px, width_px, steps,
+                                  guidance, seed, latent_out, stream);
+}
+
+lens_status lens_sample_euler_masked(lens_dit* h, const uint16_t* txt_cond, const int* len_cond,
+                                     const uint16_t* txt_uncond, const int* len_uncond, int B, int n_txt,
+                                     int height_px, int width_px, int steps, float guidance, uint64_t seed,
+                                     float* latent_out, void* stream) {
   if (!h || !latent_out || (n_txt > 0 && !txt_cond)) return LENS_ERR_INVALID_ARG;
   if (steps < 1 || !isfinite(guidance)) return LENS_ERR_INVALID_ARG;
   if (height_px <= 0 || width_px <= 0 || height_px % 16 || width_px % 16) return LENS_ERR_SHAPE;
@@ -867,14 +893,32 @@ lens_status lens_sample_euler(lens_dit* h, const uint16_t* txt_cond, const uint1
   if (s) return s;
   if (B < 1) return LENS_ERR_SHAPE;
   cudaStream_t st = (cudaStream_t)stream;
-  if (!cfg) txt_uncond = nullptr;
+  if (!cfg) {
+    txt_uncond = nullptr;
+    len_uncond = nullptr;
+  }
+  // valid text lengths of the forward rows: cond rows, then uncond rows
+  const bool masked = len_cond || len_uncond;
+  TextLengths tl;
+  if (masked) {
+    if (Bf > kMaxRows) return LENS_ERR_SHAPE;
+    for (int b = 0; b < B; ++b) {
+      const int lc = len_cond ? len_cond[b] : n_txt, lu = len_uncond ? len_uncond[b] : n_txt;
+      if (lc < 0 || lc > n_txt || lu < 0 || lu > n_txt) return LENS_ERR_SHAPE;
+      tl.n[b] = lc;
+      if (cfg) tl.n[B + b] = lu;
+    }
+  }
+  const TextLengths* tlp = masked ? &tl : nullptr;
   // On a created stream the call is captured once as a CUDA graph and replayed
   // while the arguments stay the same (the legacy default stream cannot capture).
-  if (st == nullptr) return enqueue_sample(h, txt_cond, txt_uncond, B, n_txt, gh, gw, steps, guidance, seed, latent_out, st);
+  if (st == nullptr)
+    return enqueue_sample(h, txt_cond, txt_uncond, B, n_txt, gh, gw, steps, guidance, seed, latent_out, tlp, st);
   lens_dit::SampleGraph& g = h->sg;
   if (g.valid && g.txt_cond == txt_cond && g.txt_uncond == txt_uncond && g.latent_out == latent_out &&
       g.stream == st && g.B == B && g.n_txt == n_txt && g.height_px == height_px && g.width_px == width_px &&
-      g.steps == steps && g.guidance == guidance && g.seed == seed && g.prof_kind == h->prof_kind) {
+      g.steps == steps && g.guidance == guidance && g.seed == seed && g.prof_kind == h->prof_kind &&
+      g.masked == masked && (!masked || memcmp(g.lens.n, tl.n, sizeof(int) * Bf) == 0)) {
     LENS_CUDA(cudaGraphLaunch(g.exec, st));
     h->launches += g.launches;
     return LENS_OK;
@@ -882,7 +926,7 @@ lens_status lens_sample_euler(lens_dit* h, const uint16_t* txt_cond, const uint1
   drop_sample_graph(h);
   const int64_t l0 = h->launches;
   if (cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return LENS_ERR_CUDA;
-  s = enqueue_sample(h, txt_cond, txt_uncond, B, n_txt, gh, gw, steps, guidance, seed, latent_out, st);
+  s = enqueue_sample(h, txt_cond, txt_uncond, B, n_txt, gh, gw, steps, guidance, seed, latent_out, tlp, st);
   cudaGraph_t graph = nullptr;
   const cudaError_t ce = cudaStreamEndCapture(st, &graph);
   if (s != LENS_OK || ce != cudaSuccess) {
@@ -908,6 +952,8 @@ lens_status lens_sample_euler(lens_dit* h, const uint16_t* txt_cond, const uint1
   g.guidance = guidance;
   g.seed = seed;
   g.prof_kind = h->prof_kind;
+  g.masked = masked;
+  g.lens = tl;
   g.graph = graph;
   g.exec = exec;
   g.launches = h->launches - l0;
@@ -1041,7 +1087,21 @@ lens_status lens_op_gemm_bf16(const uint16_t* A, const uint16_t* Bm, const float
 
 lens_status lens_op_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int n_txt, int n_img,
                               uint16_t* out_txt, uint16_t* out_img, void* stream) {
+  return lens_op_attention_masked(q, k, v, B, n_txt, n_img, nullptr, out_txt, out_img, stream);
+}
+
+lens_status lens_op_attention_masked(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int n_txt,
+                                     int n_img, const int* txt_len, uint16_t* out_txt, uint16_t* out_img,
+                                     void* stream) {
   if (!q || !k || !v || (n_txt > 0 && !out_txt) || (n_img > 0 && !out_img)) return LENS_ERR_INVALID_ARG;
+  TextLengths tl;
+  if (txt_len) {
+    if (B > kMaxRows) return LENS_ERR_SHAPE;
+    for (int b = 0; b < B; ++b) {
+      if (txt_len[b] < 0 || txt_len[b] > n_txt) return LENS_ERR_SHAPE;
+      tl.n[b] = txt_len[b];
+    }
+  }
   if (B < 1 || n_txt < 0 || n_img < 0 || n_txt + n_img < 1) return LENS_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15)
     return LENS_ERR_INVALID_ARG;
@@ -1050,7 +1110,7 @@ lens_status lens_op_attention(const uint16_t* q, const uint16_t* k, const uint16
   LENS_CUDA(launch_joint_attention(
       reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k),
       reinterpret_cast<const __nv_bfloat16*>(v), B, kHeads, n_txt, n_img, reinterpret_cast<__nv_bfloat16*>(out_txt),
-      reinterpret_cast<__nv_bfloat16*>(out_img), err, (cudaStream_t)stream));
+      reinterpret_cast<__nv_bfloat16*>(out_img), txt_len ? &tl : nullptr, err, (cudaStream_t)stream));
   return LENS_OK;
 }
 

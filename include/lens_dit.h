@@ -124,6 +124,16 @@ LENS_API lens_status lens_dit_forward(lens_dit* h, const float* img_tokens, int 
                              const uint16_t* txt, int n_txt, const float* t, float* v_out,
                              void* stream);
 
+/* lens_dit_forward with a text padding mask ("Lens" blog, "Exploring Text Encoder":
+ * zero-padded text tokens are masked, so the DiT never sees them): text keys at and
+ * past txt_len[b] are not attended by any query of batch row b.
+ *   txt_len  host int [B], 0 <= txt_len[b] <= n_txt, or NULL (no padding).
+ * B <= 64 when txt_len is given.  Errors as lens_dit_forward, plus SHAPE for a
+ * length out of range. */
+LENS_API lens_status lens_dit_forward_masked(lens_dit* h, const float* img_tokens, int B, int grid_h, int grid_w,
+                                             const uint16_t* txt, int n_txt, const int* txt_len, const float* t,
+                                             float* v_out, void* stream);
+
 /* Flow-matching Euler sampler ("Flow Matching 训练目标": x_t = (1-t) x0 + t x1,
  * v = x1 - x0; integrate t from 1 to 0 with `steps` uniform steps,
  * x <- x - v / steps, model input t_k = 1 - k/steps).  With guidance != 1 the
@@ -141,6 +151,17 @@ LENS_API lens_status lens_dit_forward(lens_dit* h, const float* img_tokens, int 
 LENS_API lens_status lens_sample_euler(lens_dit* h, const uint16_t* txt_cond, const uint16_t* txt_uncond,
                               int B, int n_txt, int height_px, int width_px, int steps,
                               float guidance, uint64_t seed, float* latent_out, void* stream);
+
+/* lens_sample_euler with text padding masks: len_cond / len_uncond host int [B]
+ * (valid text lengths of the conditional / unconditional features), either may be
+ * NULL for "all n_txt valid".  2B <= 64 when a length array is given.
+ * On a stream created by the caller, a call is captured as a CUDA graph and
+ * replayed while every argument stays the same (this holds for lens_sample_euler
+ * too); the legacy default stream runs the kernels directly. */
+LENS_API lens_status lens_sample_euler_masked(lens_dit* h, const uint16_t* txt_cond, const int* len_cond,
+                                              const uint16_t* txt_uncond, const int* len_uncond, int B, int n_txt,
+                                              int height_px, int width_px, int steps, float guidance, uint64_t seed,
+                                              float* latent_out, void* stream);
 
 /* Test hook: run blocks [first, last) in place on a residual stream.
  *   h_img dev fp32 [B, grid_h*grid_w, 1536], h_txt dev fp32 [B, n_txt, 1536]
@@ -201,6 +222,12 @@ LENS_API lens_status lens_op_gemm_bf16(const uint16_t* A, const uint16_t* B, con
 LENS_API lens_status lens_op_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
                               int n_txt, int n_img, uint16_t* out_txt, uint16_t* out_img,
                               void* stream);
+
+/* lens_op_attention with text padding: text keys at and past txt_len[b] (host int
+ * [B], B <= 64; NULL = none) are not attended. */
+LENS_API lens_status lens_op_attention_masked(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
+                                              int n_txt, int n_img, const int* txt_len, uint16_t* out_txt,
+                                              uint16_t* out_img, void* stream);
 
 /* Euler step with optional CFG on tokens: x -= dt * (vu + g (vc - vu)), or
  * x -= dt * vc when v_uncond is NULL.  x, v_cond, v_uncond dev fp32 [n]. */

@@ -176,15 +176,19 @@ def text_input(W: Weights, E: np.ndarray, eps: float) -> np.ndarray:
 
 
 # ============================================================ attention (a8)
-def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
-    """softmax(q k^T / sqrt(d)) v per head, no mask.  q: [B, H, Nq, d]; k, v: [B, H, N, d].
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, key_mask: Optional[np.ndarray] = None) -> np.ndarray:
+    """softmax(q k^T / sqrt(d)) v per head.  q: [B, H, Nq, d]; k, v: [B, H, N, d];
+    key_mask [B, N] (True = the key is attended) or None for no mask.
     [survey] "交叉注意力与条件注入": text and image tokens are concatenated into one
-    sequence for joint attention; [mlx] "双流注意力机制"."""
+    sequence for joint attention; [mlx] "双流注意力机制"; [blog] "Exploring Text
+    Encoder": zero-padded text tokens are masked out, so the DiT never sees them."""
     d = q.shape[-1]
     out = np.empty(q.shape[:-1] + (v.shape[-1],), dtype=np.result_type(q, v))
     for b in range(q.shape[0]):                   # heads are independent; one at a time
         for h in range(q.shape[1]):
             s = (q[b, h] @ k[b, h].T) / math.sqrt(d)
+            if key_mask is not None:
+                s = np.where(key_mask[b][None, :], s, -np.inf)
             s = s - s.max(axis=-1, keepdims=True)
             p = np.exp(s)
             p = p / p.sum(axis=-1, keepdims=True)
@@ -209,10 +213,22 @@ def gated_mlp(W: Weights, name: str, x: np.ndarray) -> np.ndarray:
     return linear(W, name + ".w2", silu(linear(W, name + ".w1", x)) * linear(W, name + ".w3", x))
 
 
+def text_key_mask(B: int, n_txt: int, n_img: int, txt_len: Optional[Sequence[int]]) -> Optional[np.ndarray]:
+    """[B, n_txt + n_img] attention key mask: text key n of sample b is attended iff
+    n < txt_len[b]; image keys always.  None (no mask) when txt_len is None.
+    READING: padding sits at the end of the text tokens ("zero-pad to the same size")."""
+    if txt_len is None:
+        return None
+    m = np.ones((B, n_txt + n_img), bool)
+    for b in range(B):
+        m[b, int(txt_len[b]):n_txt] = False
+    return m
+
+
 def block(W: Weights, i: int, h_img: np.ndarray, h_txt: np.ndarray, temb: np.ndarray,
           angles: np.ndarray, heads: int, eps: float,
-          img_rows: Optional[np.ndarray] = None, txt_rows: Optional[np.ndarray] = None
-          ) -> Tuple[np.ndarray, np.ndarray]:
+          img_rows: Optional[np.ndarray] = None, txt_rows: Optional[np.ndarray] = None,
+          txt_len: Optional[Sequence[int]] = None) -> Tuple[np.ndarray, np.ndarray]:
     """One dual-stream MMDiT block on h_img [B, Ni, D], h_txt [B, Nt, D], temb [B, D].
 
     Each stream: AdaLN-modulated RMSNorm, its own fused QKV, per-head QK-RMSNorm
@@ -225,7 +241,8 @@ def block(W: Weights, i: int, h_img: np.ndarray, h_txt: np.ndarray, temb: np.nda
     the pre-modulation RMSNorm; the gates multiply the branch output.
 
     img_rows / txt_rows select the query rows whose outputs are wanted (all when None);
-    keys and values always cover every token.  Returns the selected rows.
+    keys and values always cover every token.  txt_len [B] masks text keys at and past
+    each sample's valid length (padding).  Returns the selected rows.
     """
     p = f"transformer_blocks.{i}."
     B, Ni, D = h_img.shape
@@ -250,7 +267,7 @@ def block(W: Weights, i: int, h_img: np.ndarray, h_txt: np.ndarray, temb: np.nda
     ir = np.arange(Ni) if img_rows is None else np.asarray(img_rows)
     tr = np.arange(Nt) if txt_rows is None else np.asarray(txt_rows)
     q_sel = np.concatenate([tr, Nt + ir])
-    O = _unheads(attention(Q[:, :, q_sel, :], K, V))
+    O = _unheads(attention(Q[:, :, q_sel, :], K, V, text_key_mask(B, Nt, Ni, txt_len)))
     O_txt, O_img = O[:, :len(tr)], O[:, len(tr):]
 
     hi = h_img[:, ir] + g1i * linear(W, p + "attn.to_out", O_img)
@@ -272,9 +289,11 @@ def final_layer(W: Weights, h_img: np.ndarray, temb: np.ndarray, eps: float) -> 
 
 # ============================================================ whole forward
 def forward(W: Weights, dims, X: np.ndarray, grid_h: int, grid_w: int, E: np.ndarray,
-            t: Sequence[float], blocks: Optional[int] = None) -> np.ndarray:
+            t: Sequence[float], blocks: Optional[int] = None,
+            txt_len: Optional[Sequence[int]] = None) -> np.ndarray:
     """Velocity v [B, Ni, 128] of the denoiser for tokens X [B, Ni, 128], text
-    features E [B, Nt, 4, 2880] and per-sample timesteps t [B]."""
+    features E [B, Nt, 4, 2880] (valid lengths txt_len [B], None = all valid) and
+    per-sample timesteps t [B]."""
     n_blocks = dims.num_blocks if blocks is None else blocks
     dt = W.dtype
     temb = timestep_embedding(W, np.asarray(t, F64), dims.freq_dim)
@@ -282,7 +301,7 @@ def forward(W: Weights, dims, X: np.ndarray, grid_h: int, grid_w: int, E: np.nda
     h_txt = text_input(W, upcast(E, dt), dims.eps)
     ang = rope_angles(position_ids(grid_h, grid_w, E.shape[1]), dims.rope_axes, dims.rope_theta)
     for i in range(n_blocks):
-        h_img, h_txt = block(W, i, h_img, h_txt, temb, ang, dims.heads, dims.eps)
+        h_img, h_txt = block(W, i, h_img, h_txt, temb, ang, dims.heads, dims.eps, txt_len=txt_len)
     return final_layer(W, h_img, temb, dims.eps)
 
 
@@ -351,22 +370,29 @@ def sample_euler(velocity: Callable[[np.ndarray, float, bool], np.ndarray], x1: 
 
 def sample(W: Weights, dims, E_cond: np.ndarray, E_uncond: Optional[np.ndarray], B: int,
            grid_h: int, grid_w: int, steps: int, guidance: float, seed: int,
-           blocks: Optional[int] = None) -> np.ndarray:
+           blocks: Optional[int] = None, len_cond: Optional[Sequence[int]] = None,
+           len_uncond: Optional[Sequence[int]] = None) -> np.ndarray:
     """Full sampler: seeded noise latent [B, 32, 2h, 2w] -> latent at t = 0.
     Cond and uncond run as one batch of 2B (cond first) when guidance != 1.
-    READING: unconditional text = zeros of the same shape when E_uncond is None."""
+    READING: unconditional text = zeros of the same shape when E_uncond is None.
+    len_cond / len_uncond: valid text lengths per sample (None = all valid)."""
     C, p = dims.latent_channels, dims.patch
     z = noise(seed, B * C * p * grid_h * p * grid_w).reshape(B, C, p * grid_h, p * grid_w)
     x = z.astype(W.dtype)
     if guidance != 1.0 and E_uncond is None:
         E_uncond = np.zeros_like(E_cond)
+    Nt = E_cond.shape[1]
+    lc = None if len_cond is None and len_uncond is None else \
+        list(len_cond if len_cond is not None else [Nt] * B)
+    lu = None if lc is None else list(len_uncond if len_uncond is not None else [Nt] * B)
     for t in timesteps(steps):
         X = patchify(x, p)
         if guidance == 1.0:
-            v = forward(W, dims, X, grid_h, grid_w, E_cond, [t] * B, blocks)
+            v = forward(W, dims, X, grid_h, grid_w, E_cond, [t] * B, blocks, txt_len=lc)
         else:
             vv = forward(W, dims, np.concatenate([X, X]), grid_h, grid_w,
-                         np.concatenate([E_cond, E_uncond]), [t] * (2 * B), blocks)
+                         np.concatenate([E_cond, E_uncond]), [t] * (2 * B), blocks,
+                         txt_len=None if lc is None else lc + lu)
             v = cfg_combine(vv[:B], vv[B:], guidance)
         x = euler(x, unpatchify(v, grid_h, grid_w, C, p), 1.0 / steps)
     return x

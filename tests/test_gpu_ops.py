@@ -146,3 +146,24 @@ def test_euler_cfg_op():
     L.lens_op_euler_cfg(xd, dev(vc), None, n, 0.5, 1.0)
     _sync()
     assert np.allclose(host(xd), x - 0.5 * vc, rtol=1e-6, atol=1e-6)
+
+
+@pytest.mark.parametrize("B,nt,ni,lens", [(2, 16, 64, [5, 16]), (2, 256, 1024, [0, 200]), (3, 130, 333, [129, 1, 64])])
+def test_joint_attention_text_padding(B, nt, ni, lens):
+    """Text keys at and past each row's valid length are masked (length 0 masks
+    whole key tiles before any valid key is seen)."""
+    import torch
+    rng = np.random.default_rng(nt + ni)
+    N = nt + ni
+    q, k, v = (f32_to_bf16_bits(rng.standard_normal((B, 24, N, 64)).astype(np.float32) * s) for s in (1.5, 1.5, 1))
+    ot = torch.full((B, nt, 1536), -1, dtype=torch.int16, device="cuda")
+    oi = torch.full((B, ni, 1536), -1, dtype=torch.int16, device="cuda")
+    L.lens_op_attention_masked(dev(q), dev(k), dev(v), B, nt, ni, lens, ot, oi)
+    _sync()
+    heads = 24 if N <= 600 else 4
+    mask = o.text_key_mask(B, nt, ni, lens)
+    ref = o.attention(bf16_to_f64(q)[:, :heads], bf16_to_f64(k)[:, :heads], bf16_to_f64(v)[:, :heads], mask)
+    ref = ref.transpose(0, 2, 1, 3).reshape(B, N, heads * 64)
+    got = np.concatenate([bf16_to_f64(host(ot)), bf16_to_f64(host(oi))], axis=1)[..., :heads * 64]
+    assert np.all(np.isfinite(got))
+    assert cos_sim(got, ref) > 0.9999 and rel_l2(got, ref) < 1e-2

@@ -359,3 +359,35 @@ def test_box_muller_closed_form():
         u2 = (int(w2[i]) >> 11) / 2.0 ** 53
         assert 0.0 < u1 <= 1.0 and 0.0 <= u2 < 1.0
         assert z[i] == np.float32(math.sqrt(-2 * math.log(u1)) * math.cos(2 * math.pi * u2))
+
+
+# ------------------------------------------------------------------ text padding mask
+def test_masked_attention_brute_force_and_no_influence():
+    rng = np.random.default_rng(12)
+    q, k, v = (rng.standard_normal((2, 2, 6, 4)) for _ in range(3))
+    mask = o.text_key_mask(2, 3, 3, [1, 3])        # sample 0 keeps 1 of 3 text keys
+    out = o.attention(q, k, v, mask)
+    for b in range(2):
+        keep = np.where(mask[b])[0]
+        for h in range(2):
+            assert np.allclose(out[b, h], _attn_loops(q[b, h], k[b, h][keep], v[b, h][keep]), atol=1e-12)
+    k2, v2 = k.copy(), v.copy()
+    k2[0, :, 1:3] = 1e3 * rng.standard_normal((2, 2, 4))   # change only masked keys / values
+    v2[0, :, 1:3] = -7.0
+    assert np.allclose(o.attention(q, k2, v2, mask), out, atol=1e-12)
+    assert np.allclose(o.attention(q, k, v, o.text_key_mask(2, 3, 3, [3, 3])), o.attention(q, k, v), atol=1e-12)
+    assert o.text_key_mask(2, 3, 3, None) is None
+
+
+def test_block_padding_has_no_influence(tinyW):
+    h_img, h_txt, temb = _block_inputs(TINY, Ni=6, Nt=4)
+    ang = o.rope_angles(o.position_ids(2, 3, 4), TINY.rope_axes, TINY.rope_theta)
+    hi, ht = o.block(tinyW, 0, h_img, h_txt, temb, ang, TINY.heads, TINY.eps, txt_len=[2, 4])
+    h_txt2 = h_txt.copy()
+    h_txt2[0, 2:] = 50.0 * np.random.default_rng(13).standard_normal((2, TINY.hidden))
+    hi2, ht2 = o.block(tinyW, 0, h_img, h_txt2, temb, ang, TINY.heads, TINY.eps, txt_len=[2, 4])
+    assert np.allclose(hi2, hi, atol=1e-10) and np.allclose(ht2[:, :2], ht[:, :2], atol=1e-10)
+    assert np.allclose(ht2[1], ht[1], atol=1e-10)
+    # the unpadded sample equals the unmasked block
+    hu, tu = o.block(tinyW, 0, h_img, h_txt, temb, ang, TINY.heads, TINY.eps)
+    assert np.allclose(hi[1], hu[1], atol=1e-12) and not np.allclose(hi[0], hu[0], atol=1e-6)
