@@ -20,6 +20,34 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+
+// Packed fp32 pairs (Blackwell f32x2 arithmetic): one instruction for two lanes
+// of the softmax's scale-and-shift and running sums.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// three-input maximum (one instruction on sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ============================================================ tcgen05 version
 // One CTA per (256 query rows = two 128-row tiles X = 0, 1; head; batch row).
 // Warp roles (320 threads):
@@ -219,13 +247,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < 128; ++i)
           if (j * BKV + i >= txt_valid && j * BKV + i < txt_pad_end) sc[i] = -INFINITY;
       }
-      // 8 independent partial maxima / sums keep the dependency chains short
+      // 8 independent partial maxima (three-input max) keep the dependency chains short
       float pm[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) pm[q] = sc[q];
+      for (int q = 0; q < 8; ++q) {
+        pm[q] = max3f(sc[q], sc[q + 8], sc[q + 16]);
 #pragma unroll
-      for (int i = 8; i < 128; ++i) pm[i & 7] = fmaxf(pm[i & 7], sc[i]);
-      float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+        for (int t = 3; t < 15; t += 2) pm[q] = max3f(pm[q], sc[q + 8 * t], sc[q + 8 * t + 8]);
+        pm[q] = fmaxf(pm[q], sc[q + 120]);
+      }
+      float mx = max3f(max3f(pm[0], pm[1], pm[2]), max3f(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
       mx *= scale_log2;
       float corr = 1.f;
       if (mx > m + kRescaleThreshold) {
@@ -234,16 +265,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // every key seen so far masked: m is still -inf and so is every score here
       const float m_base = m == -INFINITY ? 0.f : m;
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+      // x = s log2(e) / 8 - m for two keys per instruction
+      const uint64_t sl2 = f2_pack(scale_log2, scale_log2), mb2 = f2_pack(-m_base, -m_base);
       uint32_t pk[64];
 #pragma unroll
       for (int i = 0; i < 128; i += 2) {
-        const float e0 = ex2(fmaf(sc[i], scale_log2, -m_base));
-        const float e1 = ex2(fmaf(sc[i + 1], scale_log2, -m_base));
-        ps[i & 7] += e0;
-        ps[(i + 1) & 7] += e1;
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(sc[i], sc[i + 1]), sl2, mb2), x0, x1);
+        const float e0 = ex2(x0), e1 = ex2(x1);
+        acc2[(i >> 1) & 3] = f2_add(acc2[(i >> 1) & 3], f2_pack(e0, e1));
         pk[i >> 1] = pack_bf16x2(e0, e1);
       }
+      float ps[8];
+      f2_unpack(acc2[0], ps[0], ps[1]);
+      f2_unpack(acc2[1], ps[2], ps[3]);
+      f2_unpack(acc2[2], ps[4], ps[5]);
+      f2_unpack(acc2[3], ps[6], ps[7]);
       const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       l = l * corr + rs;
       if (j > 0) {
