@@ -10,10 +10,11 @@ weights as raw bit patterns and upcasts them itself.
 Sources (page title, section):
   [blog]    "Lens" blog post (zjwfufu.github.io), sections "Overview" (block arithmetic:
             48 blocks, hidden 1536, 24 heads, gate/up/down 1536x4096, AdaLN 1536x9216,
-            dual stream), "Exploring Image Editing" (CFG combination).
+            dual stream), "Exploring Image Editing" (CFG combination; "norm-rescaled").
   [paper]   "Lens: 重新思考基础文生图模型的训练效率" summary page, sections "前置知识 /
-            Flow Matching 训练目标" (x_t = (1-t) x0 + t x1, v = x1 - x0) and
-            "方法步骤详情" (RMSNorm + RoPE dual stream; 20 steps CFG 5.0; Turbo 4 steps).
+            Flow Matching 训练目标" (x_t = (1-t) x0 + t x1, v = x1 - x0; mu(n) linear
+            interpolation of the timestep schedule by resolution) and "方法步骤详情"
+            (RMSNorm + RoPE dual stream; mu = 1.06 at 512^2; 20 steps CFG 5.0; Turbo 4).
   [mlx]     "深入 Lens-Turbo-3.8B-bf16 内核" article, sections "核心规格一览", "双流注意力机制",
             "自适应调制与 RMSNorm", "3D RoPE 旋转位置编码", "多层级文本特征融合",
             "Patchify 补丁化与输出投影", "guidance 1.0".
@@ -349,6 +350,50 @@ def timesteps(steps: int) -> np.ndarray:
     return 1.0 - np.arange(steps, dtype=F64) / steps
 
 
+def cfg_rescaled(v_cond: np.ndarray, v_uncond: np.ndarray, scale: float, phi: float) -> np.ndarray:
+    """Norm-rescaled CFG.  [blog] "Exploring Image Editing" names Lens's guidance
+    "norm-rescaled CFG" and says it drives the difference of two guided velocities
+    towards zero, but prints only u + s (c - u).  READING: form the plain combination
+    v = u + s (c - u), then pull its L2 norm back to the conditional one,
+        v <- phi * v * |c| / |v| + (1 - phi) * v,
+    with each norm taken over one sample's whole velocity (every axis but the first).
+    phi = 0 is plain CFG, phi = 1 the full rescale; |v| = 0 leaves v unchanged."""
+    v = cfg_combine(v_cond, v_uncond, scale)
+    axes = tuple(range(1, v.ndim))
+    nc = np.sqrt(np.sum(v_cond.astype(F64) ** 2, axis=axes, keepdims=True))
+    nv = np.sqrt(np.sum(v.astype(F64) ** 2, axis=axes, keepdims=True))
+    r = np.where(nv > 0, nc / np.where(nv > 0, nv, 1.0), 1.0)
+    return phi * r * v + (1.0 - phi) * v
+
+
+def time_shift(t, mu: float):
+    """Resolution shift of a flow-matching time, t' = e^mu t / (e^mu t + 1 - t).
+    [paper] "Flow Matching 训练目标" ties the timestep schedule at each resolution to
+    a mu(n) "linear interpolation" and [paper] "方法步骤详情" gives mu = 1.06 for the
+    512^2 stage, but no formula is printed.  READING: the exponential shift of the
+    published flow-matching schedule (Esser et al. 2024, resolution-dependent
+    shifting of timestep schedules), with e^mu the shift factor: t = 0 and t = 1
+    stay fixed, mu = 0 is the identity, mu > 0 spends more of the steps near t = 1."""
+    t = np.asarray(t, dtype=F64)
+    a = np.exp(F64(mu))
+    return a * t / (a * t + (1.0 - t))
+
+
+def shift_mu(n_img_tokens: int, n1: int, mu1: float, n2: int, mu2: float) -> float:
+    """mu linear in the image token count n through (n1, mu1) and (n2, mu2) ([paper]
+    "Flow Matching 训练目标": mu(n) is a linear interpolation).  The pages give one
+    point only: 512^2 (32 x 32 = 1024 tokens) at mu = 1.06; the other anchor is the
+    caller's."""
+    return float(mu1 + (mu2 - mu1) * (n_img_tokens - n1) / (n2 - n1))
+
+
+def time_grid(steps: int, mu: Optional[float] = None) -> np.ndarray:
+    """t_0 .. t_S (S + 1 values): the uniform grid 1 - k/S, shifted by time_shift(., mu)
+    when mu is given.  Step k feeds the model t_k and moves by t_k - t_{k+1}."""
+    t = 1.0 - np.arange(steps + 1, dtype=F64) / steps
+    return t if mu is None else time_shift(t, mu)
+
+
 def euler(x: np.ndarray, v: np.ndarray, dt: float) -> np.ndarray:
     """x_{t-dt} = x_t - dt * v.  [paper] "Flow Matching 训练目标": x_t = (1-t) x0 + t x1
     with v = x1 - x0, so integrating from t = 1 (noise) to t = 0 (data) subtracts v."""
@@ -356,26 +401,37 @@ def euler(x: np.ndarray, v: np.ndarray, dt: float) -> np.ndarray:
 
 
 def sample_euler(velocity: Callable[[np.ndarray, float, bool], np.ndarray], x1: np.ndarray,
-                 steps: int, guidance: float) -> np.ndarray:
-    """Integrate from t = 1 to 0 with S uniform Euler steps.  velocity(x, t, cond) gives
-    the conditional (cond=True) or unconditional prediction.  guidance == 1 evaluates
-    the conditional model only ([mlx] "guidance 1.0": no doubled forward)."""
+                 steps: int, guidance: float, mu: Optional[float] = None, phi: float = 0.0) -> np.ndarray:
+    """Integrate from t = 1 to 0 with S Euler steps.  velocity(x, t, cond) gives the
+    conditional (cond=True) or unconditional prediction.  guidance == 1 evaluates the
+    conditional model only ([mlx] "guidance 1.0": no doubled forward).  mu shifts the
+    time grid (time_grid), phi rescales the guided velocity (cfg_rescaled); with
+    neither, the steps are the uniform 1/S."""
     x = x1
-    for t in timesteps(steps):
-        vc = velocity(x, float(t), True)
-        v = vc if guidance == 1.0 else cfg_combine(vc, velocity(x, float(t), False), guidance)
-        x = euler(x, v, 1.0 / steps)
+    tg = time_grid(steps, mu)
+    for k in range(steps):
+        t = float(tg[k])
+        dt = 1.0 / steps if mu is None else float(tg[k] - tg[k + 1])
+        vc = velocity(x, t, True)
+        if guidance == 1.0:
+            v = vc
+        else:
+            vu = velocity(x, t, False)
+            v = cfg_combine(vc, vu, guidance) if phi == 0.0 else cfg_rescaled(vc, vu, guidance, phi)
+        x = euler(x, v, dt)
     return x
 
 
 def sample(W: Weights, dims, E_cond: np.ndarray, E_uncond: Optional[np.ndarray], B: int,
            grid_h: int, grid_w: int, steps: int, guidance: float, seed: int,
            blocks: Optional[int] = None, len_cond: Optional[Sequence[int]] = None,
-           len_uncond: Optional[Sequence[int]] = None) -> np.ndarray:
+           len_uncond: Optional[Sequence[int]] = None, mu: Optional[float] = None,
+           phi: float = 0.0) -> np.ndarray:
     """Full sampler: seeded noise latent [B, 32, 2h, 2w] -> latent at t = 0.
     Cond and uncond run as one batch of 2B (cond first) when guidance != 1.
     READING: unconditional text = zeros of the same shape when E_uncond is None.
-    len_cond / len_uncond: valid text lengths per sample (None = all valid)."""
+    len_cond / len_uncond: valid text lengths per sample (None = all valid).
+    mu: shifted time grid (time_grid); phi: norm-rescaled CFG (cfg_rescaled)."""
     C, p = dims.latent_channels, dims.patch
     z = noise(seed, B * C * p * grid_h * p * grid_w).reshape(B, C, p * grid_h, p * grid_w)
     x = z.astype(W.dtype)
@@ -385,7 +441,10 @@ def sample(W: Weights, dims, E_cond: np.ndarray, E_uncond: Optional[np.ndarray],
     lc = None if len_cond is None and len_uncond is None else \
         list(len_cond if len_cond is not None else [Nt] * B)
     lu = None if lc is None else list(len_uncond if len_uncond is not None else [Nt] * B)
-    for t in timesteps(steps):
+    tg = time_grid(steps, mu)
+    for k in range(steps):
+        t = float(tg[k])
+        dt = 1.0 / steps if mu is None else float(tg[k] - tg[k + 1])
         X = patchify(x, p)
         if guidance == 1.0:
             v = forward(W, dims, X, grid_h, grid_w, E_cond, [t] * B, blocks, txt_len=lc)
@@ -393,8 +452,9 @@ def sample(W: Weights, dims, E_cond: np.ndarray, E_uncond: Optional[np.ndarray],
             vv = forward(W, dims, np.concatenate([X, X]), grid_h, grid_w,
                          np.concatenate([E_cond, E_uncond]), [t] * (2 * B), blocks,
                          txt_len=None if lc is None else lc + lu)
-            v = cfg_combine(vv[:B], vv[B:], guidance)
-        x = euler(x, unpatchify(v, grid_h, grid_w, C, p), 1.0 / steps)
+            v = cfg_combine(vv[:B], vv[B:], guidance) if phi == 0.0 else \
+                cfg_rescaled(vv[:B], vv[B:], guidance, phi)
+        x = euler(x, unpatchify(v, grid_h, grid_w, C, p), dt)
     return x
 
 

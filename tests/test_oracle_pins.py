@@ -328,6 +328,80 @@ def test_cfg_special_scales():
     assert calls.count(False) == 0                        # guidance 1: no unconditional pass
 
 
+# ------------------------------------------------------------------ sampler variants
+def test_time_shift_fixed_points_values_and_group():
+    t = np.linspace(0.0, 1.0, 11)
+    assert np.array_equal(o.time_shift(t, 0.0), t)                 # mu = 0: identity
+    for mu in (-1.3, 0.4, 1.06, 2.5):
+        assert o.time_shift(0.0, mu) == 0.0 and o.time_shift(1.0, mu) == 1.0
+        assert np.all(np.diff(o.time_shift(t, mu)) > 0)          # order of the grid kept
+    # shift factor 3 (mu = ln 3), worked by hand: 1/2 -> 3/4, 1/4 -> 1/2, 1/10 -> 1/4
+    assert abs(o.time_shift(0.5, math.log(3.0)) - 0.75) < 1e-15
+    assert abs(o.time_shift(0.25, math.log(3.0)) - 0.5) < 1e-15
+    assert abs(o.time_shift(0.1, math.log(3.0)) - 0.25) < 1e-15
+    # shifts compose by adding mu (e^mu is the factor, not mu), and -mu undoes mu
+    assert np.allclose(o.time_shift(o.time_shift(t, 0.7), -0.25), o.time_shift(t, 0.45), atol=1e-14)
+    assert np.allclose(o.time_shift(o.time_shift(t, 1.06), -1.06), t, atol=1e-14)
+    # mu > 0 moves every inner time towards the noise end t = 1
+    assert np.all(o.time_shift(t[1:-1], 1.06) > t[1:-1])
+
+
+def test_shift_mu_is_linear_through_both_anchors():
+    # the pages' one anchor: 512^2 -> 32 x 32 = 1024 tokens at mu = 1.06
+    assert o.shift_mu(1024, 1024, 1.06, 4096, 1.5) == pytest.approx(1.06, abs=1e-15)
+    assert o.shift_mu(4096, 1024, 1.06, 4096, 1.5) == pytest.approx(1.5, abs=1e-15)
+    assert o.shift_mu(2560, 1024, 1.06, 4096, 1.5) == pytest.approx(1.28, abs=1e-15)   # midpoint
+    assert o.shift_mu(8100, 1024, 1.06, 4096, 1.06) == pytest.approx(1.06, abs=1e-15)  # flat line
+
+
+def test_time_grid_uniform_and_shifted():
+    assert o.time_grid(4).tolist() == [1.0, 0.75, 0.5, 0.25, 0.0]
+    g = o.time_grid(7, 1.06)
+    assert g[0] == 1.0 and g[-1] == 0.0 and len(g) == 8
+    dt = -np.diff(g)
+    assert np.all(dt > 0) and abs(dt.sum() - 1.0) < 1e-15         # steps telescope to 1
+    assert dt[0] < 1.0 / 7 < dt[-1]                               # small steps near noise
+
+
+def test_sampler_on_shifted_grid_worked_by_hand():
+    # v(x, t) = x: Euler multiplies by (1 - dt_k).  S = 2, mu = ln 3: t = 1, 3/4, 0,
+    # dt = 1/4, 3/4, so x -> x (3/4)(1/4) and the model sees t = 1 then t = 3/4
+    seen = []
+    vel = lambda x, t, c: (seen.append(t), x)[1]
+    x = o.sample_euler(vel, np.full(3, 2.0), 2, 1.0, mu=math.log(3.0))
+    assert np.allclose(x, 2.0 * 0.75 * 0.25, atol=1e-15)
+    assert seen == pytest.approx([1.0, 0.75], abs=1e-15)
+    # straight paths stay exact on any grid whose steps sum to 1
+    rng = np.random.default_rng(12)
+    x0, x1 = rng.standard_normal((2, 3, 8))
+    assert np.allclose(o.sample_euler(lambda x, t, c: x1 - x0, x1, 5, 1.0, mu=1.3), x0, atol=1e-12)
+
+
+def test_cfg_rescaled_values_and_invariants():
+    # by hand: c = (3, 4), u = 0, s = 2 -> plain (6, 8), |c| = 5, |plain| = 10
+    c = np.array([[3.0, 4.0]])
+    u = np.zeros((1, 2))
+    assert np.allclose(o.cfg_rescaled(c, u, 2.0, 1.0), [[3.0, 4.0]], atol=1e-15)
+    assert np.allclose(o.cfg_rescaled(c, u, 2.0, 0.5), [[4.5, 6.0]], atol=1e-15)
+    rng = np.random.default_rng(13)
+    c, u = rng.standard_normal((2, 3, 4, 5))
+    assert np.array_equal(o.cfg_rescaled(c, u, 5.0, 0.0), o.cfg_combine(c, u, 5.0))   # phi = 0: plain
+    assert np.allclose(o.cfg_rescaled(c, u, 1.0, 1.0), c, atol=1e-14)                 # s = 1: cond
+    v, p = o.cfg_rescaled(c, u, 5.0, 1.0), o.cfg_combine(c, u, 5.0)
+    for b in range(3):                                  # per sample: |v| = |c|, same direction
+        assert np.linalg.norm(v[b]) == pytest.approx(np.linalg.norm(c[b]), rel=1e-13)
+        cosv = np.sum(v[b] * p[b]) / (np.linalg.norm(v[b]) * np.linalg.norm(p[b]))
+        assert cosv == pytest.approx(1.0, abs=1e-13)
+    c2 = c.copy()
+    c2[1] *= 7.0
+    assert np.array_equal(o.cfg_rescaled(c2, u, 5.0, 1.0)[0], v[0])   # samples are independent
+    z = np.zeros((2, 6))
+    assert np.array_equal(o.cfg_rescaled(z, z, 5.0, 1.0), z)          # zero velocity stays zero
+    # inside the sampler: c = 1, u = 3 (4 elements): plain -7, rescaled to norm 2 -> -1
+    vel = lambda x, t, cond: np.full_like(x, 1.0 if cond else 3.0)
+    assert np.allclose(o.sample_euler(vel, np.zeros(4), 2, 5.0, phi=1.0), 1.0, atol=1e-15)
+
+
 # ------------------------------------------------------------------ noise
 def test_splitmix64_published_vectors():
     want = [int(r[0], 16) for r in _golden("splitmix64_seed0.txt")]
