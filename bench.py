@@ -2,8 +2,9 @@
 """Throughput of the Lens MMDiT denoiser + flow-matching Euler sampler on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload turbo_1024] [--impl lens|reference]
+                    [--cfg-rescale PHI] [--shift-mu MU]
 
-One step = one `lens_sample_euler` call on seeded synthetic inputs: noise, text
+One step = one `lens_sample_euler_ex` call on seeded synthetic inputs: noise, text
 input head, timestep/AdaLN modulation for every step, S denoiser forwards of 48
 blocks, Euler (+CFG) updates and unpatchify.  Default workload: Turbo-style
 4-step sampling at 1024^2 (4096 image + 256 text tokens, batch 1, guidance 1).
@@ -15,6 +16,8 @@ CUDA events on the launching stream, max over ranks.  The 8.2 GB of weights are
 streamed by every forward, so the working set is far larger than L2 (126 MB).
 Multi-GPU (torchrun): independent replicas, one sample stream per GPU, no data
 exchange (weak scaling).  --impl reference times the CPU oracle instead.
+--cfg-rescale / --shift-mu time the sampler variants (norm-rescaled CFG, shifted
+time grid); without them the call is the plain sampler.
 """
 from __future__ import annotations
 
@@ -249,6 +252,10 @@ def main():
     ap.add_argument("--workload", default="turbo_1024", choices=[k for k, v in WORKLOADS.items() if v.steps > 0])
     ap.add_argument("--impl", default="lens", choices=["lens", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cfg-rescale", type=float, default=0.0,
+                    help="norm-rescaled CFG weight phi in [0, 1] (0: plain CFG)")
+    ap.add_argument("--shift-mu", type=float, default=None,
+                    help="shifted time grid with this mu (default: uniform grid)")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -259,6 +266,8 @@ def main():
               "forward_rows": wl.batch * (2 if wl.guidance != 1.0 else 1),
               "l2": "inputs larger than L2: 8.2 GB of weights streamed by every forward",
               "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+    if args.cfg_rescale != 0.0 or args.shift_mu is not None:
+        config["sampler_variant"] = {"cfg_rescale": args.cfg_rescale, "shift_mu": args.shift_mu}
 
     if args.impl == "reference":
         if rank != 0:
@@ -294,9 +303,17 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
     out = torch.empty((wl.batch, 32, 2 * wl.grid_h, 2 * wl.grid_w), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
+    opt = L.lens_sampler_default_options()
+    opt.guidance, opt.cfg_rescale = wl.guidance, args.cfg_rescale
+    if args.shift_mu is not None:
+        opt.time_shift, opt.shift_mu = 1, args.shift_mu
+
+    def sample(text):
+        L.lens_sample_euler_ex(h, text, None, None, None, wl.batch, wl.n_txt, wl.height_px, wl.width_px, wl.steps,
+                               opt, seed, out)
+
     def step():
-        L.lens_sample_euler(h, txt, None, wl.batch, wl.n_txt, wl.height_px, wl.width_px, wl.steps, wl.guidance,
-                            seed, out)
+        sample(txt)
 
     for _ in range(args.warmup):
         step()
@@ -329,14 +346,12 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
     txt_dev = torch.empty_like(txt)
     for _ in range(2):
         txt_dev.copy_(txt_pinned, non_blocking=True)
-        L.lens_sample_euler(h, txt_dev, None, wl.batch, wl.n_txt, wl.height_px, wl.width_px, wl.steps, wl.guidance,
-                            seed, out)
+        sample(txt_dev)
         out_pinned.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
     def e2e_step():
         txt_dev.copy_(txt_pinned, non_blocking=True)
-        L.lens_sample_euler(h, txt_dev, None, wl.batch, wl.n_txt, wl.height_px, wl.width_px, wl.steps, wl.guidance,
-                            seed, out)
+        sample(txt_dev)
         out_pinned.copy_(out, non_blocking=True)
 
     e2e_ms = timed_region(e2e_step, args.steps, barrier, torch.cuda.synchronize, EventTimer(stream))

@@ -26,7 +26,8 @@ EXPORTS = [
     "lens_op_attention", "lens_op_euler_cfg", "lens_dit_op_timestep", "lens_dit_op_text_input",
     "lens_device_sm_count", "lens_dit_profile_kernel", "lens_dit_profile_read", "lens_dit_launch_count",
     "lens_op_timestep_embed_noalloc", "lens_dit_forward_masked", "lens_sample_euler_masked",
-    "lens_op_attention_masked",
+    "lens_op_attention_masked", "lens_sampler_default_options", "lens_shift_mu", "lens_time_grid",
+    "lens_sample_euler_ex", "lens_dit_op_euler_cfg_rescaled",
 ]
 
 KERNELS = {"none": 0, "attention": 1, "gemm_qkv": 2, "gemm_out": 3, "gemm_w13": 4, "gemm_w2": 5, "rmsnorm_mod": 6,
@@ -46,6 +47,11 @@ class lens_dit_config(ctypes.Structure):
                 ("txt_dim", ctypes.c_int), ("rope_axes", ctypes.c_int * 3), ("rope_theta", ctypes.c_float),
                 ("eps", ctypes.c_float), ("freq_dim", ctypes.c_int), ("max_batch", ctypes.c_int),
                 ("max_img_tokens", ctypes.c_int), ("max_txt_tokens", ctypes.c_int), ("max_timesteps", ctypes.c_int)]
+
+
+class lens_sampler_options(ctypes.Structure):
+    _fields_ = [("guidance", ctypes.c_float), ("cfg_rescale", ctypes.c_float), ("time_shift", ctypes.c_int),
+                ("shift_mu", ctypes.c_float)]
 
 
 class lens_weight(ctypes.Structure):
@@ -93,6 +99,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lens_dit_forward_masked": (I, [P, P, I, I, I, P, I, P, P, P, P]),
         "lens_sample_euler_masked": (I, [P, P, P, P, P, I, I, I, I, I, F, U64, P, P]),
         "lens_op_attention_masked": (I, [P, P, P, I, I, I, P, P, P, P]),
+        "lens_sampler_default_options": (I, [ctypes.POINTER(lens_sampler_options)]),
+        "lens_shift_mu": (ctypes.c_double, [I, I, ctypes.c_double, I, ctypes.c_double]),
+        "lens_time_grid": (I, [I, I, ctypes.c_double, P]),
+        "lens_sample_euler_ex": (I, [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(lens_sampler_options), U64, P,
+                                     P]),
+        "lens_dit_op_euler_cfg_rescaled": (I, [P, P, P, P, I, L, F, F, F, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -206,6 +218,38 @@ def lens_sample_euler_masked(h: LensDit, txt_cond, len_cond, txt_uncond, len_unc
     _check(load_library().lens_sample_euler_masked(h.ptr, _ptr(txt_cond), _iptr(lc), _ptr(txt_uncond), _iptr(lu), B,
                                                    n_txt, height_px, width_px, steps, guidance, seed,
                                                    _ptr(latent_out), _stream(stream)), "lens_sample_euler_masked")
+
+
+def lens_sampler_default_options() -> lens_sampler_options:
+    o = lens_sampler_options()
+    _check(load_library().lens_sampler_default_options(ctypes.byref(o)), "lens_sampler_default_options")
+    return o
+
+
+def lens_shift_mu(n_img_tokens: int, n1: int, mu1: float, n2: int, mu2: float) -> float:
+    return load_library().lens_shift_mu(n_img_tokens, n1, mu1, n2, mu2)
+
+
+def lens_time_grid(steps: int, time_shift: bool, mu: float) -> np.ndarray:
+    t = np.empty(max(steps, 0) + 1, dtype=np.float64)
+    _check(load_library().lens_time_grid(steps, 1 if time_shift else 0, mu, t.ctypes.data), "lens_time_grid")
+    return t
+
+
+def lens_sample_euler_ex(h: LensDit, txt_cond, len_cond, txt_uncond, len_uncond, B: int, n_txt: int,
+                         height_px: int, width_px: int, steps: int, opt: lens_sampler_options, seed: int,
+                         latent_out, stream=None) -> None:
+    lc, lu = _ints(len_cond), _ints(len_uncond)
+    _check(load_library().lens_sample_euler_ex(h.ptr, _ptr(txt_cond), _iptr(lc), _ptr(txt_uncond), _iptr(lu), B,
+                                               n_txt, height_px, width_px, steps, ctypes.byref(opt), seed,
+                                               _ptr(latent_out), _stream(stream)), "lens_sample_euler_ex")
+
+
+def lens_dit_op_euler_cfg_rescaled(h: LensDit, x, v_cond, v_uncond, B: int, per_sample: int, dt: float,
+                                   guidance: float, phi: float, stream=None) -> None:
+    _check(load_library().lens_dit_op_euler_cfg_rescaled(h.ptr, _ptr(x), _ptr(v_cond), _ptr(v_uncond), B, per_sample,
+                                                         dt, guidance, phi, _stream(stream)),
+           "lens_dit_op_euler_cfg_rescaled")
 
 
 def lens_sample_euler(h: LensDit, txt_cond, txt_uncond, B: int, n_txt: int, height_px: int, width_px: int,

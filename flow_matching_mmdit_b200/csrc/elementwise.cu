@@ -369,6 +369,110 @@ cudaError_t launch_small_linear(const float* x, int T, int K, const __nv_bfloat1
                                                        silu_rows);
   return cudaGetLastError();
 }
+// ------------------------------------------------------------------ norm-rescaled CFG (a14 variant)
+// v = f * p with p = u + g (c - u) and f = phi |c| / |p| + (1 - phi), both norms over
+// one sample's whole velocity.  Pass 1 writes per-block partial sums of c^2 and p^2
+// (fp64) to fixed slots; pass 2 reduces a sample's slots in a fixed order (so the
+// result never depends on scheduling) and applies the Euler update.
+__global__ void cfg_norm_partials_kernel(const float* __restrict__ vc, const float* __restrict__ vu,
+                                         int64_t per_sample, float g, double* __restrict__ part) {
+  const int b = blockIdx.y;
+  const float* c = vc + (int64_t)b * per_sample;
+  const float* u = vu + (int64_t)b * per_sample;
+  float sc = 0.f, sp = 0.f;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < per_sample;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const float cv = c[e], uv = u[e];
+    const float pv = fmaf(g, cv - uv, uv);
+    sc = fmaf(cv, cv, sc);
+    sp = fmaf(pv, pv, sp);
+  }
+  double dc = sc, dp = sp;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    dc += __shfl_xor_sync(0xffffffffu, dc, o);
+    dp += __shfl_xor_sync(0xffffffffu, dp, o);
+  }
+  __shared__ double red[2][32];
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    red[0][w] = dc;
+    red[1][w] = dp;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double a = 0.0, q = 0.0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+      a += red[0][i];
+      q += red[1][i];
+    }
+    double* dst = part + ((int64_t)b * gridDim.x + blockIdx.x) * 2;
+    dst[0] = a;
+    dst[1] = q;
+  }
+}
+
+__global__ void euler_cfg_rescaled_kernel(float* __restrict__ x, const float* __restrict__ vc,
+                                          const float* __restrict__ vu, int64_t per_sample, int64_t total,
+                                          float dt, float g, float phi, const double* __restrict__ part,
+                                          int nparts, __nv_bfloat16* __restrict__ xin) {
+  const int b = blockIdx.y;
+  __shared__ float s_f;
+  if (threadIdx.x < 32) {
+    // lane l sums slots l, l + 32, ...; then a fixed xor tree
+    double a = 0.0, q = 0.0;
+    for (int i = threadIdx.x; i < nparts; i += 32) {
+      a += part[((int64_t)b * nparts + i) * 2];
+      q += part[((int64_t)b * nparts + i) * 2 + 1];
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      a += __shfl_xor_sync(0xffffffffu, a, o);
+      q += __shfl_xor_sync(0xffffffffu, q, o);
+    }
+    if (threadIdx.x == 0) s_f = (float)((double)phi * (q > 0.0 ? sqrt(a / q) : 1.0) + (1.0 - (double)phi));
+  }
+  __syncthreads();
+  const float f = s_f;
+  const int64_t base = (int64_t)b * per_sample;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < per_sample;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = base + i;
+    const float cv = vc[e], uv = vu[e];
+    const float xn = x[e] - dt * (f * fmaf(g, cv - uv, uv));
+    x[e] = xn;
+    if (xin) {      // refresh the [hi | lo] img_in operand of the cond and the uncond row
+      const __nv_bfloat16 hi = __float2bfloat16_rn(xn);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(xn - __bfloat162float(hi));
+      const int64_t row = e >> 7;
+      const int ft = (int)(e & 127);
+      xin[row * 256 + ft] = hi;
+      xin[row * 256 + 128 + ft] = lo;
+      xin[(row + (total >> 7)) * 256 + ft] = hi;
+      xin[(row + (total >> 7)) * 256 + 128 + ft] = lo;
+    }
+  }
+}
+
+cudaError_t launch_cfg_norm_partials(const float* vc, const float* vu, int64_t per_sample, int B, float guidance,
+                                     double* part, cudaStream_t st) {
+  if (per_sample <= 0 || B <= 0) return cudaSuccess;
+  cfg_norm_partials_kernel<<<dim3(kCfgNormParts, B), 256, 0, st>>>(vc, vu, per_sample, guidance, part);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_euler_cfg_rescaled(float* x, const float* vc, const float* vu, int64_t per_sample, int B,
+                                      float dt, float guidance, float phi, const double* part, __nv_bfloat16* xin,
+                                      cudaStream_t st) {
+  if (per_sample <= 0 || B <= 0) return cudaSuccess;
+  if (xin && (per_sample & 127)) return cudaErrorInvalidValue;
+  int64_t blocks = (per_sample + 256 * 8 - 1) / (256 * 8);
+  if (blocks > 1024) blocks = 1024;
+  euler_cfg_rescaled_kernel<<<dim3((unsigned)blocks, B), 256, 0, st>>>(x, vc, vu, per_sample, per_sample * B, dt,
+                                                                       guidance, phi, part, kCfgNormParts, xin);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_euler_cfg(float* x, const float* v, int64_t per_sample, int B, bool cfg, float dt,
                              float guidance, __nv_bfloat16* xin, cudaStream_t st) {
   const int64_t n = per_sample * B;

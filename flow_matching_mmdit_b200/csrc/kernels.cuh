@@ -70,5 +70,14 @@ cudaError_t launch_euler_cfg(float* x, const float* v, int64_t per_sample, int B
                              float guidance, __nv_bfloat16* xin, cudaStream_t st);
 cudaError_t launch_euler_plain(float* x, const float* vc, const float* vu, int64_t n, float dt, float guidance,
                                cudaStream_t st);
+// norm-rescaled CFG: pass 1 writes kCfgNormParts x 2 fp64 partial norms per sample to
+// `part` ([B][kCfgNormParts][2]); pass 2 reduces them and applies
+// x -= dt (phi |c| / |p| + 1 - phi) p, p = u + g (c - u), refreshing xin when given
+constexpr int kCfgNormParts = 128;
+cudaError_t launch_cfg_norm_partials(const float* vc, const float* vu, int64_t per_sample, int B, float guidance,
+                                     double* part, cudaStream_t st);
+cudaError_t launch_euler_cfg_rescaled(float* x, const float* vc, const float* vu, int64_t per_sample, int B,
+                                      float dt, float guidance, float phi, const double* part, __nv_bfloat16* xin,
+                                      cudaStream_t st);
 
 }  // namespace lens

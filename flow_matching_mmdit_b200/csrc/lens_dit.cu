@@ -79,6 +79,7 @@ struct lens_dit {
   __nv_bfloat16 *xin, *a_img, *a_txt, *q, *k, *v, *o_img, *o_txt, *u_img, *u_txt, *txt_cat, *stemb;
   float *h_img, *h_txt, *h_txt0, *vtok, *xtok, *tfeat, *hid, *temb, *mod;
   float2* rope;
+  double* cfgpart;     // per-sample partial norms of the norm-rescaled CFG
   int* err;
   // the last sampler call, captured as a CUDA graph and replayed for identical calls
   struct SampleGraph {
@@ -86,7 +87,8 @@ struct lens_dit {
     const void *txt_cond, *txt_uncond, *latent_out;
     cudaStream_t stream;
     int B, n_txt, height_px, width_px, steps;
-    float guidance;
+    float guidance, cfg_rescale, shift_mu;
+    int time_shift;
     uint64_t seed;
     int prof_kind;
     bool masked;
@@ -439,6 +441,7 @@ static size_t layout_workspace(lens_dit* h, Bump& b) {
   h->temb = b.take<float>((size_t)kMaxTimesteps * kHidden);
   h->mod = b.take<float>(Tm * h->modw);
   h->rope = b.take<float2>(N * 32);
+  h->cfgpart = b.take<double>(Bm * kCfgNormParts * 2);
   h->err = b.take<int>(1);
   return b.off;
 }
@@ -677,11 +680,27 @@ static void drop_sample_graph(lens_dit* h) {
   h->sg = lens_dit::SampleGraph();
 }
 
+// t_0 .. t_S of the sampler: the uniform grid 1 - k/S, optionally mapped through the
+// resolution shift t' = e^mu t / (e^mu t + 1 - t) (summary page "Lens: 重新思考基础文生图
+// 模型的训练效率", "Flow Matching 训练目标": the schedule at each resolution follows a
+// mu(n) linear interpolation; the published resolution-dependent shift is taken).
+static void sampler_time_grid(int steps, bool shift, double mu, double* t) {
+  const double a = exp(mu);
+  for (int k = 0; k <= steps; ++k) {
+    const double u = 1.0 - (double)k / (double)steps;
+    t[k] = shift ? a * u / (a * u + (1.0 - u)) : u;
+  }
+  t[steps] = 0.0;
+}
+
 // Enqueue one sampler call on `st` (validated arguments).
 static lens_status enqueue_sample(lens_dit* h, const uint16_t* txt_cond, const uint16_t* txt_uncond, int B,
-                                  int n_txt, int gh, int gw, int steps, float guidance, uint64_t seed,
+                                  int n_txt, int gh, int gw, int steps, const lens_sampler_options& o, uint64_t seed,
                                   float* latent_out, const TextLengths* tl, cudaStream_t st) {
+  const float guidance = o.guidance;
   const bool cfg = guidance != 1.0f;
+  const bool rescale = cfg && o.cfg_rescale != 0.0f;
+  const bool shift = o.time_shift != 0;
   const int Ni = gh * gw;
   const int Bf = cfg ? 2 * B : B;
   const int64_t per_sample = (int64_t)Ni * kInCh;
@@ -693,14 +712,25 @@ static lens_status enqueue_sample(lens_dit* h, const uint16_t* txt_cond, const u
   if ((s = text_in_gemm(h, Bf * n_txt, h->h_txt0, st))) return s;
 
   const int chunk = h->cfg.max_timesteps;
+  std::vector<double> grid(steps + 1);
+  sampler_time_grid(steps, shift, o.shift_mu, grid.data());
   float tv[kMaxTimesteps];
   for (int k0 = 0; k0 < steps; k0 += chunk) {
     const int T = steps - k0 < chunk ? steps - k0 : chunk;
-    for (int j = 0; j < T; ++j) tv[j] = (float)(1.0 - (double)(k0 + j) / (double)steps);
+    for (int j = 0; j < T; ++j) tv[j] = (float)grid[k0 + j];
     if ((s = compute_modulation(h, tv, T, st))) return s;
     for (int j = 0; j < T; ++j) {
+      // uniform grid: every step is exactly 1/S, as in the plain sampler
+      const float dt = shift ? (float)(grid[k0 + j] - grid[k0 + j + 1]) : 1.0f / (float)steps;
       if ((s = run_forward_core(h, Bf, gh, gw, n_txt, h->mod + (int64_t)j * h->modw, 0, h->vtok, tl, st))) return s;
-      LENS_LAUNCH(h, 0, st, launch_euler_cfg(h->xtok, h->vtok, per_sample, B, cfg, 1.0f / (float)steps, guidance, h->xin, st));
+      if (rescale) {
+        const float* vu = h->vtok + (int64_t)B * per_sample;
+        LENS_LAUNCH(h, 0, st, launch_cfg_norm_partials(h->vtok, vu, per_sample, B, guidance, h->cfgpart, st));
+        LENS_LAUNCH(h, 0, st, launch_euler_cfg_rescaled(h->xtok, h->vtok, vu, per_sample, B, dt, guidance,
+                                                        o.cfg_rescale, h->cfgpart, h->xin, st));
+      } else {
+        LENS_LAUNCH(h, 0, st, launch_euler_cfg(h->xtok, h->vtok, per_sample, B, cfg, dt, guidance, h->xin, st));
+      }
     }
   }
   LENS_LAUNCH(h, 0, st, launch_unpatchify(h->xtok, B, gh, gw, latent_out, st));
@@ -883,8 +913,43 @@ lens_status lens_sample_euler_masked(lens_dit* h, const uint16_t* txt_cond, cons
                                      const uint16_t* txt_uncond, const int* len_uncond, int B, int n_txt,
                                      int height_px, int width_px, int steps, float guidance, uint64_t seed,
                                      float* latent_out, void* stream) {
-  if (!h || !latent_out || (n_txt > 0 && !txt_cond)) return LENS_ERR_INVALID_ARG;
+  lens_sampler_options o;
+  lens_sampler_default_options(&o);
+  o.guidance = guidance;
+  return lens_sample_euler_ex(h, txt_cond, len_cond, txt_uncond, len_uncond, B, n_txt, height_px, width_px, steps,
+                              &o, seed, latent_out, stream);
+}
+
+lens_status lens_sampler_default_options(lens_sampler_options* o) {
+  if (!o) return LENS_ERR_INVALID_ARG;
+  o->guidance = 1.0f;
+  o->cfg_rescale = 0.0f;
+  o->time_shift = 0;
+  o->shift_mu = 0.0f;
+  return LENS_OK;
+}
+
+double lens_shift_mu(int n_img_tokens, int n1, double mu1, int n2, double mu2) {
+  if (n1 == n2) return NAN;
+  return mu1 + (mu2 - mu1) * (double)(n_img_tokens - n1) / (double)(n2 - n1);
+}
+
+lens_status lens_time_grid(int steps, int time_shift, double mu, double* t_out) {
+  if (!t_out || steps < 1 || !isfinite(mu) || fabs(mu) > 50.0) return LENS_ERR_INVALID_ARG;
+  sampler_time_grid(steps, time_shift != 0, mu, t_out);
+  return LENS_OK;
+}
+
+lens_status lens_sample_euler_ex(lens_dit* h, const uint16_t* txt_cond, const int* len_cond,
+                                 const uint16_t* txt_uncond, const int* len_uncond, int B, int n_txt, int height_px,
+                                 int width_px, int steps, const lens_sampler_options* opt, uint64_t seed,
+                                 float* latent_out, void* stream) {
+  if (!h || !opt || !latent_out || (n_txt > 0 && !txt_cond)) return LENS_ERR_INVALID_ARG;
+  const float guidance = opt->guidance;
   if (steps < 1 || !isfinite(guidance)) return LENS_ERR_INVALID_ARG;
+  if (!(opt->cfg_rescale >= 0.0f && opt->cfg_rescale <= 1.0f) || !isfinite(opt->shift_mu) ||
+      fabsf(opt->shift_mu) > 50.0f)
+    return LENS_ERR_INVALID_ARG;
   if (height_px <= 0 || width_px <= 0 || height_px % 16 || width_px % 16) return LENS_ERR_SHAPE;
   const bool cfg = guidance != 1.0f;
   const int gh = height_px / 16, gw = width_px / 16;
@@ -913,11 +978,13 @@ lens_status lens_sample_euler_masked(lens_dit* h, const uint16_t* txt_cond, cons
   // On a created stream the call is captured once as a CUDA graph and replayed
   // while the arguments stay the same (the legacy default stream cannot capture).
   if (st == nullptr)
-    return enqueue_sample(h, txt_cond, txt_uncond, B, n_txt, gh, gw, steps, guidance, seed, latent_out, tlp, st);
+    return enqueue_sample(h, txt_cond, txt_uncond, B, n_txt, gh, gw, steps, *opt, seed, latent_out, tlp, st);
   lens_dit::SampleGraph& g = h->sg;
   if (g.valid && g.txt_cond == txt_cond && g.txt_uncond == txt_uncond && g.latent_out == latent_out &&
       g.stream == st && g.B == B && g.n_txt == n_txt && g.height_px == height_px && g.width_px == width_px &&
-      g.steps == steps && g.guidance == guidance && g.seed == seed && g.prof_kind == h->prof_kind &&
+      g.steps == steps && g.guidance == guidance && g.cfg_rescale == opt->cfg_rescale &&
+      g.time_shift == (opt->time_shift != 0) && g.shift_mu == opt->shift_mu && g.seed == seed &&
+      g.prof_kind == h->prof_kind &&
       g.masked == masked && (!masked || memcmp(g.lens.n, tl.n, sizeof(int) * Bf) == 0)) {
     LENS_CUDA(cudaGraphLaunch(g.exec, st));
     h->launches += g.launches;
@@ -926,7 +993,7 @@ lens_status lens_sample_euler_masked(lens_dit* h, const uint16_t* txt_cond, cons
   drop_sample_graph(h);
   const int64_t l0 = h->launches;
   if (cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return LENS_ERR_CUDA;
-  s = enqueue_sample(h, txt_cond, txt_uncond, B, n_txt, gh, gw, steps, guidance, seed, latent_out, tlp, st);
+  s = enqueue_sample(h, txt_cond, txt_uncond, B, n_txt, gh, gw, steps, *opt, seed, latent_out, tlp, st);
   cudaGraph_t graph = nullptr;
   const cudaError_t ce = cudaStreamEndCapture(st, &graph);
   if (s != LENS_OK || ce != cudaSuccess) {
@@ -950,6 +1017,9 @@ lens_status lens_sample_euler_masked(lens_dit* h, const uint16_t* txt_cond, cons
   g.width_px = width_px;
   g.steps = steps;
   g.guidance = guidance;
+  g.cfg_rescale = opt->cfg_rescale;
+  g.time_shift = opt->time_shift != 0;
+  g.shift_mu = opt->shift_mu;
   g.seed = seed;
   g.prof_kind = h->prof_kind;
   g.masked = masked;
@@ -1111,6 +1181,18 @@ lens_status lens_op_attention_masked(const uint16_t* q, const uint16_t* k, const
       reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k),
       reinterpret_cast<const __nv_bfloat16*>(v), B, kHeads, n_txt, n_img, reinterpret_cast<__nv_bfloat16*>(out_txt),
       reinterpret_cast<__nv_bfloat16*>(out_img), txt_len ? &tl : nullptr, err, (cudaStream_t)stream));
+  return LENS_OK;
+}
+
+lens_status lens_dit_op_euler_cfg_rescaled(lens_dit* h, float* x, const float* v_cond, const float* v_uncond, int B,
+                                           int64_t per_sample, float dt, float guidance, float phi, void* stream) {
+  if (!h || !x || !v_cond || !v_uncond) return LENS_ERR_INVALID_ARG;
+  if (!isfinite(dt) || !isfinite(guidance) || !(phi >= 0.0f && phi <= 1.0f)) return LENS_ERR_INVALID_ARG;
+  if (B < 1 || B > h->cfg.max_batch || per_sample < 1) return LENS_ERR_SHAPE;
+  cudaStream_t st = (cudaStream_t)stream;
+  LENS_LAUNCH(h, 0, st, launch_cfg_norm_partials(v_cond, v_uncond, per_sample, B, guidance, h->cfgpart, st));
+  LENS_LAUNCH(h, 0, st, launch_euler_cfg_rescaled(x, v_cond, v_uncond, per_sample, B, dt, guidance, phi, h->cfgpart,
+                                                  nullptr, st));
   return LENS_OK;
 }
 

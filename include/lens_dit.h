@@ -163,6 +163,53 @@ LENS_API lens_status lens_sample_euler_masked(lens_dit* h, const uint16_t* txt_c
                                               int height_px, int width_px, int steps, float guidance, uint64_t seed,
                                               float* latent_out, void* stream);
 
+/* Sampler variants (plain value struct, filled by lens_sampler_default_options).
+ *   guidance     CFG scale s; 1 evaluates the conditional model only.
+ *   cfg_rescale  phi in [0, 1], used when guidance != 1: the guided velocity
+ *                p = u + s (c - u) becomes (phi |c| / |p| + 1 - phi) p, both L2
+ *                norms over one sample's whole velocity; |p| = 0 leaves p as is.
+ *                Blog "Lens", section "Exploring Image Editing": Lens runs a
+ *                "norm-rescaled CFG" (only u + s (c - u) is printed; this rescale
+ *                toward the conditional norm is the reading taken).  0 = plain CFG.
+ *   time_shift   nonzero: the uniform grid u_k = 1 - k/S is mapped through
+ *                t_k = e^mu u_k / (e^mu u_k + 1 - u_k).  Summary page "Lens:
+ *                重新思考基础文生图模型的训练效率", section "Flow Matching 训练目标":
+ *                the timestep schedule at each resolution follows a mu(n) linear
+ *                interpolation (section "方法步骤详情": mu = 1.06 at 512^2); the
+ *                formula is not printed, the published resolution-dependent shift
+ *                is taken.  Step k feeds the model t_k and moves by t_k - t_{k+1}.
+ *   shift_mu     mu of the shift, |mu| <= 50 (see lens_shift_mu). */
+typedef struct {
+  float guidance;
+  float cfg_rescale;
+  int time_shift;
+  float shift_mu;
+} lens_sampler_options;
+
+/* Defaults: guidance 1, cfg_rescale 0, time_shift 0, shift_mu 0 (the plain sampler).
+ * Errors: INVALID_ARG for NULL. */
+LENS_API lens_status lens_sampler_default_options(lens_sampler_options* opt);
+
+/* mu(n) linear in the image token count n through (n1, mu1) and (n2, mu2).  The
+ * pages give one point (512^2 = 1024 tokens: mu = 1.06); the second anchor is the
+ * caller's.  Host only; returns NaN when n1 == n2. */
+LENS_API double lens_shift_mu(int n_img_tokens, int n1, double mu1, int n2, double mu2);
+
+/* The sampler's time grid t_0 .. t_steps (host double [steps + 1], caller-owned),
+ * uniform or shifted as in lens_sampler_options.  Host only.
+ * Errors: INVALID_ARG (NULL, steps < 1, non-finite mu or |mu| > 50). */
+LENS_API lens_status lens_time_grid(int steps, int time_shift, double mu, double* t_out);
+
+/* lens_sample_euler_masked with the variants of `opt` (host, not kept).  Arguments
+ * and graph replay as lens_sample_euler_masked; the options are part of what must
+ * stay the same for a replay.
+ * Errors: as lens_sample_euler_masked, plus INVALID_ARG for a NULL opt,
+ * cfg_rescale outside [0, 1] or |shift_mu| > 50 (or not finite). */
+LENS_API lens_status lens_sample_euler_ex(lens_dit* h, const uint16_t* txt_cond, const int* len_cond,
+                                          const uint16_t* txt_uncond, const int* len_uncond, int B, int n_txt,
+                                          int height_px, int width_px, int steps, const lens_sampler_options* opt,
+                                          uint64_t seed, float* latent_out, void* stream);
+
 /* Test hook: run blocks [first, last) in place on a residual stream.
  *   h_img dev fp32 [B, grid_h*grid_w, 1536], h_txt dev fp32 [B, n_txt, 1536]
  *   t host fp32 [B].  Errors as lens_dit_forward, plus SHAPE for a bad range. */
@@ -233,6 +280,16 @@ LENS_API lens_status lens_op_attention_masked(const uint16_t* q, const uint16_t*
  * x -= dt * vc when v_uncond is NULL.  x, v_cond, v_uncond dev fp32 [n]. */
 LENS_API lens_status lens_op_euler_cfg(float* x, const float* v_cond, const float* v_uncond, int64_t n,
                               float dt, float guidance, void* stream);
+
+/* Euler step with norm-rescaled CFG (see lens_sampler_options.cfg_rescale) on B
+ * samples of per_sample values each: x -= dt (phi |c| / |p| + 1 - phi) p with
+ * p = u + guidance (c - u), norms per sample.  x, v_cond, v_uncond dev fp32
+ * [B, per_sample].  Uses the handle's workspace, so calls on one handle must not
+ * overlap.  Errors: INVALID_ARG (NULL, non-finite dt or guidance, phi outside
+ * [0, 1]), SHAPE (B < 1, B > max_batch, per_sample < 1). */
+LENS_API lens_status lens_dit_op_euler_cfg_rescaled(lens_dit* h, float* x, const float* v_cond,
+                                                    const float* v_uncond, int B, int64_t per_sample, float dt,
+                                                    float guidance, float phi, void* stream);
 
 /* Handle ops: the timestep embedding temb [T, 1536] (dev fp32) of host t[T], and
  * the AdaLN modulation of every block plus norm_out for those timesteps,

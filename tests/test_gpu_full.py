@@ -43,10 +43,11 @@ def test_forward_48_blocks_512(full):
     assert c >= 0.995
 
 
-def _composed(h, Ec, B, gh, gw, nt, steps, guidance, seed, gpu_euler=False):
+def _composed(h, Ec, B, gh, gw, nt, steps, guidance, seed, gpu_euler=False, mu=None, phi=0.0):
     """Oracle Euler/CFG loop whose velocity field is the library's forward.  With
     gpu_euler the update runs through the library's fp32 Euler/CFG op instead of
-    the oracle's fp64 one, so the two sides round identically."""
+    the oracle's fp64 one, so the two sides round identically.  mu / phi select the
+    shifted grid and the norm-rescaled CFG."""
     Ni = gh * gw
     x = torch.empty((B, Ni, 128), dtype=torch.float32, device="cuda")
     L.lens_op_noise_tokens(seed, B, gh, gw, x)
@@ -55,17 +56,24 @@ def _composed(h, Ec, B, gh, gw, nt, steps, guidance, seed, gpu_euler=False):
     E = torch.cat([Ec, torch.zeros_like(Ec)]) if cfg else Ec
     rows = 2 * B if cfg else B
     v = torch.empty((rows, Ni, 128), dtype=torch.float32, device="cuda")
-    for t in o.timesteps(steps):
+    grid = o.time_grid(steps, mu)
+    for k in range(steps):
+        t = grid[k]
+        dt = 1.0 / steps if mu is None else float(np.float32(grid[k] - grid[k + 1]))
         xin = np.concatenate([xk, xk]) if cfg else xk
         L.lens_dit_forward(h, dev(xin.astype(np.float32)), rows, gh, gw, E, nt, [float(np.float32(t))] * rows, v)
         if gpu_euler:
             xd = dev(xk.astype(np.float32))
-            L.lens_op_euler_cfg(xd, v[:B], v[B:] if cfg else None, xd.numel(), 1.0 / steps, guidance)
+            if cfg and phi != 0.0:
+                L.lens_dit_op_euler_cfg_rescaled(h, xd, v[:B], v[B:], B, Ni * 128, dt, guidance, phi)
+            else:
+                L.lens_op_euler_cfg(xd, v[:B], v[B:] if cfg else None, xd.numel(), dt, guidance)
             xk = host(xd).astype(np.float64)
             continue
         vv = host(v).astype(np.float64)
-        vel = o.cfg_combine(vv[:B], vv[B:], guidance) if cfg else vv
-        xk = o.euler(xk, vel, 1.0 / steps)
+        vel = vv if not cfg else (o.cfg_combine(vv[:B], vv[B:], guidance) if phi == 0.0 else
+                                  o.cfg_rescaled(vv[:B], vv[B:], guidance, phi))
+        xk = o.euler(xk, vel, dt)
         xk = xk.astype(np.float32).astype(np.float64)      # the sampler keeps its state in fp32
     return o.unpatchify(xk, gh, gw, 32)
 
@@ -91,4 +99,33 @@ def test_sampler_is_euler_over_forward(full, name, steps):
     ref = _composed(h, Ec, B, wl.grid_h, wl.grid_w, wl.n_txt, steps, wl.guidance, wl.seed)
     c, r = cos_sim(got, ref), rel_l2(got, ref)
     print(f"{name}: sampler vs composed forwards: cosine {c:.9f}, rel L2 {r:.3e}")
+    assert c >= 0.99 and r < 5e-2
+
+
+@pytest.mark.parametrize("name,steps,phi,shift", [("turbo_1024", 4, 0.0, True), ("cfg_1024", 2, 1.0, True),
+                                                  ("cfg_1440", 2, 1.0, False)])
+def test_sampler_variants_are_euler_over_forward(full, name, steps, phi, shift):
+    """Shifted grid (mu from the pages' 512^2 anchor and a 1.15 anchor at 4096
+    tokens) and norm-rescaled CFG at full sizes, checked as for the plain sampler."""
+    w, h = full
+    wl = WORKLOADS[name]
+    B = 1
+    mu = L.lens_shift_mu(wl.grid_h * wl.grid_w, 1024, 1.06, 4096, 1.15) if shift else None
+    opt = L.lens_sampler_default_options()
+    opt.guidance, opt.cfg_rescale = wl.guidance, phi
+    if shift:
+        opt.time_shift, opt.shift_mu = 1, mu
+    mu32 = None if mu is None else float(np.float32(mu))
+    Ec = dev(text_features(B, wl.n_txt, wl.seed))
+    out = torch.empty((B, 32, 2 * wl.grid_h, 2 * wl.grid_w), dtype=torch.float32, device="cuda")
+    L.lens_sample_euler_ex(h, Ec, None, None, None, B, wl.n_txt, wl.height_px, wl.width_px, steps, opt, wl.seed, out)
+    L.lens_dit_sync(h)
+    got = host(out)
+    assert np.all(np.isfinite(got))
+    same = _composed(h, Ec, B, wl.grid_h, wl.grid_w, wl.n_txt, steps, wl.guidance, wl.seed, gpu_euler=True,
+                     mu=mu32, phi=phi)
+    assert rel_l2(got, same) < 1e-6, rel_l2(got, same)
+    ref = _composed(h, Ec, B, wl.grid_h, wl.grid_w, wl.n_txt, steps, wl.guidance, wl.seed, mu=mu32, phi=phi)
+    c, r = cos_sim(got, ref), rel_l2(got, ref)
+    print(f"{name} variant (phi {phi}, shift {shift}): cosine {c:.9f}, rel L2 {r:.3e}")
     assert c >= 0.99 and r < 5e-2

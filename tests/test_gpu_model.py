@@ -283,3 +283,85 @@ def test_sampler_text_padding(small):
     ref = o.sample(o.Weights(w), d, Ec, None, B, gh, gw, 3, 5.0, seed, len_cond=[9], len_uncond=[0])
     got = host(out)
     assert cos_sim(got, ref) >= 0.99 and rel_l2(got, ref) <= 5e-2, (cos_sim(got, ref), rel_l2(got, ref))
+
+
+# ------------------------------------------------------------------ sampler variants
+@pytest.mark.parametrize("B,per,phi", [(3, 128 * 37, 0.0), (3, 128 * 37, 0.5), (3, 128 * 37, 1.0),
+                                       (2, 4096 * 128, 1.0), (1, 128, 0.25)])
+def test_euler_cfg_rescaled_op(small, B, per, phi):
+    """Norm-rescaled CFG + Euler against the oracle: per-sample norms over every
+    value of the sample, so samples with different scales must not mix."""
+    d, w, h = small
+    rng = np.random.default_rng(31 + B)
+    x, c, u = (rng.standard_normal((B, per)).astype(np.float32) for _ in range(3))
+    u[-1] *= 3.0
+    c[0] *= 0.2
+    xd = dev(x)
+    L.lens_dit_op_euler_cfg_rescaled(h, xd, dev(c), dev(u), B, per, 0.0625, 5.0, phi)
+    _sync(h)
+    ref = o.euler(x.astype(np.float64), o.cfg_rescaled(c.astype(np.float64), u.astype(np.float64), 5.0, phi), 0.0625)
+    err = np.max(np.abs(host(xd) - ref))
+    assert err <= 2e-5 * np.max(np.abs(ref)), err
+
+
+def test_euler_cfg_rescaled_edge_cases(small):
+    d, w, h = small
+    B, per = 2, 256
+    x = np.arange(B * per, dtype=np.float32).reshape(B, per) / 7.0
+    z = np.zeros((B, per), np.float32)
+    xd = dev(x)
+    L.lens_dit_op_euler_cfg_rescaled(h, xd, dev(z), dev(z), B, per, 0.5, 5.0, 1.0)   # zero velocity: no move
+    _sync(h)
+    assert np.array_equal(host(xd), x)
+    with pytest.raises(L.LensError) as e:
+        L.lens_dit_op_euler_cfg_rescaled(h, xd, dev(z), dev(z), B, per, 0.5, 5.0, 1.5)
+    assert e.value.status == 1
+    with pytest.raises(L.LensError) as e:
+        L.lens_dit_op_euler_cfg_rescaled(h, xd, dev(z), dev(z), 5, per, 0.5, 5.0, 1.0)  # > max_batch 4
+    assert e.value.status == 2
+
+
+def _options(guidance, phi, mu):
+    opt = L.lens_sampler_default_options()
+    opt.guidance, opt.cfg_rescale = guidance, phi
+    if mu is not None:
+        opt.time_shift, opt.shift_mu = 1, mu
+    return opt
+
+
+@pytest.mark.parametrize("guidance,phi,mu", [(5.0, 1.0, 1.2), (5.0, 0.5, None), (1.0, 0.0, 0.5), (4.0, 1.0, -0.3)])
+def test_sampler_variants_two_blocks(small, guidance, phi, mu):
+    d, w, h = small
+    B, gh, gw, nt, seed, steps = 2, 8, 6, 16, 99, 3
+    Ec = text_features(B, nt, 23)
+    out = torch.empty((B, 32, 2 * gh, 2 * gw), dtype=torch.float32, device="cuda")
+    L.lens_sample_euler_ex(h, dev(Ec), None, None, None, B, nt, 16 * gh, 16 * gw, steps, _options(guidance, phi, mu),
+                           seed, out)
+    _sync(h)
+    mu64 = None if mu is None else float(np.float32(mu))
+    ref = o.sample(o.Weights(w), d, Ec, None, B, gh, gw, steps, guidance, seed, mu=mu64, phi=phi)
+    got = host(out)
+    assert cos_sim(got, ref) >= 0.99 and rel_l2(got, ref) <= 5e-2, (cos_sim(got, ref), rel_l2(got, ref))
+
+
+def test_sampler_options_are_part_of_the_replay_key(small):
+    """Changing only the variant options on a created stream re-captures the graph."""
+    d, w, h = small
+    B, gh, gw, nt = 1, 8, 8, 16
+    E = dev(text_features(B, nt, 41))
+    shape = (B, 32, 2 * gh, 2 * gw)
+    plain, resc = _options(5.0, 0.0, None), _options(5.0, 1.0, 0.8)
+    refs = []
+    for opt in (plain, resc):
+        r = torch.empty(shape, dtype=torch.float32, device="cuda")
+        L.lens_sample_euler_ex(h, E, None, None, None, B, nt, 16 * gh, 16 * gw, 3, opt, 5, r)   # direct
+        _sync(h)
+        refs.append(host(r).copy())
+    assert not np.array_equal(refs[0], refs[1])
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out = torch.empty(shape, dtype=torch.float32, device="cuda")
+        for opt, want in ((plain, 0), (resc, 1), (plain, 0), (plain, 0)):
+            L.lens_sample_euler_ex(h, E, None, None, None, B, nt, 16 * gh, 16 * gw, 3, opt, 5, out)
+            L.lens_dit_sync(h, s)
+            assert np.array_equal(host(out), refs[want])
