@@ -27,7 +27,8 @@ EXPORTS = [
     "lens_device_sm_count", "lens_dit_profile_kernel", "lens_dit_profile_read", "lens_dit_launch_count",
     "lens_op_timestep_embed_noalloc", "lens_dit_forward_masked", "lens_sample_euler_masked",
     "lens_op_attention_masked", "lens_sampler_default_options", "lens_shift_mu", "lens_time_grid",
-    "lens_sample_euler_ex", "lens_dit_op_euler_cfg_rescaled",
+    "lens_sample_euler_ex", "lens_dit_op_euler_cfg_rescaled", "lens_sampler_prepare", "lens_sampler_velocity",
+    "lens_sampler_update", "lens_sampler_finish",
 ]
 
 KERNELS = {"none": 0, "attention": 1, "gemm_qkv": 2, "gemm_out": 3, "gemm_w13": 4, "gemm_w2": 5, "rmsnorm_mod": 6,
@@ -105,6 +106,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lens_sample_euler_ex": (I, [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(lens_sampler_options), U64, P,
                                      P]),
         "lens_dit_op_euler_cfg_rescaled": (I, [P, P, P, P, I, L, F, F, F, P]),
+        "lens_sampler_prepare": (I, [P, P, P, I, I, I, I, I, ctypes.POINTER(lens_sampler_options), U64, P]),
+        "lens_sampler_velocity": (I, [P, I, P, P]),
+        "lens_sampler_update": (I, [P, I, P, P, P]),
+        "lens_sampler_finish": (I, [P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -250,6 +255,26 @@ def lens_dit_op_euler_cfg_rescaled(h: LensDit, x, v_cond, v_uncond, B: int, per_
     _check(load_library().lens_dit_op_euler_cfg_rescaled(h.ptr, _ptr(x), _ptr(v_cond), _ptr(v_uncond), B, per_sample,
                                                          dt, guidance, phi, _stream(stream)),
            "lens_dit_op_euler_cfg_rescaled")
+
+
+def lens_sampler_prepare(h: LensDit, txt, txt_len, B: int, n_txt: int, height_px: int, width_px: int, steps: int,
+                         opt: lens_sampler_options, seed: int, stream=None) -> None:
+    tl = _ints(txt_len)
+    _check(load_library().lens_sampler_prepare(h.ptr, _ptr(txt), _iptr(tl), B, n_txt, height_px, width_px, steps,
+                                               ctypes.byref(opt), seed, _stream(stream)), "lens_sampler_prepare")
+
+
+def lens_sampler_velocity(h: LensDit, k: int, v_out, stream=None) -> None:
+    _check(load_library().lens_sampler_velocity(h.ptr, k, _ptr(v_out), _stream(stream)), "lens_sampler_velocity")
+
+
+def lens_sampler_update(h: LensDit, k: int, v_cond, v_uncond, stream=None) -> None:
+    _check(load_library().lens_sampler_update(h.ptr, k, _ptr(v_cond), _ptr(v_uncond), _stream(stream)),
+           "lens_sampler_update")
+
+
+def lens_sampler_finish(h: LensDit, latent_out, stream=None) -> None:
+    _check(load_library().lens_sampler_finish(h.ptr, _ptr(latent_out), _stream(stream)), "lens_sampler_finish")
 
 
 def lens_sample_euler(h: LensDit, txt_cond, txt_uncond, B: int, n_txt: int, height_px: int, width_px: int,

@@ -415,7 +415,7 @@ __global__ void cfg_norm_partials_kernel(const float* __restrict__ vc, const flo
 __global__ void euler_cfg_rescaled_kernel(float* __restrict__ x, const float* __restrict__ vc,
                                           const float* __restrict__ vu, int64_t per_sample, int64_t total,
                                           float dt, float g, float phi, const double* __restrict__ part,
-                                          int nparts, __nv_bfloat16* __restrict__ xin) {
+                                          int nparts, __nv_bfloat16* __restrict__ xin, int xin_copies) {
   const int b = blockIdx.y;
   __shared__ float s_f;
   if (threadIdx.x < 32) {
@@ -441,15 +441,17 @@ __global__ void euler_cfg_rescaled_kernel(float* __restrict__ x, const float* __
     const float cv = vc[e], uv = vu[e];
     const float xn = x[e] - dt * (f * fmaf(g, cv - uv, uv));
     x[e] = xn;
-    if (xin) {      // refresh the [hi | lo] img_in operand of the cond and the uncond row
+    if (xin) {      // refresh the [hi | lo] img_in operand of the cond (and the uncond) row
       const __nv_bfloat16 hi = __float2bfloat16_rn(xn);
       const __nv_bfloat16 lo = __float2bfloat16_rn(xn - __bfloat162float(hi));
       const int64_t row = e >> 7;
       const int ft = (int)(e & 127);
       xin[row * 256 + ft] = hi;
       xin[row * 256 + 128 + ft] = lo;
-      xin[(row + (total >> 7)) * 256 + ft] = hi;
-      xin[(row + (total >> 7)) * 256 + 128 + ft] = lo;
+      if (xin_copies == 2) {
+        xin[(row + (total >> 7)) * 256 + ft] = hi;
+        xin[(row + (total >> 7)) * 256 + 128 + ft] = lo;
+      }
     }
   }
 }
@@ -463,13 +465,39 @@ cudaError_t launch_cfg_norm_partials(const float* vc, const float* vu, int64_t p
 
 cudaError_t launch_euler_cfg_rescaled(float* x, const float* vc, const float* vu, int64_t per_sample, int B,
                                       float dt, float guidance, float phi, const double* part, __nv_bfloat16* xin,
-                                      cudaStream_t st) {
+                                      int xin_copies, cudaStream_t st) {
   if (per_sample <= 0 || B <= 0) return cudaSuccess;
   if (xin && (per_sample & 127)) return cudaErrorInvalidValue;
   int64_t blocks = (per_sample + 256 * 8 - 1) / (256 * 8);
   if (blocks > 1024) blocks = 1024;
   euler_cfg_rescaled_kernel<<<dim3((unsigned)blocks, B), 256, 0, st>>>(x, vc, vu, per_sample, per_sample * B, dt,
-                                                                       guidance, phi, part, kCfgNormParts, xin);
+                                                                       guidance, phi, part, kCfgNormParts, xin,
+                                                                       xin_copies);
+  return cudaGetLastError();
+}
+
+// One Euler step of the step-wise sampler: x -= dt (u + g (c - u)), or dt c when vu is
+// NULL, refreshing one [hi | lo] img_in operand row per token.
+__global__ void euler_step_kernel(float* __restrict__ x, const float* __restrict__ vc,
+                                  const float* __restrict__ vu, int64_t n, float dt, float g,
+                                  __nv_bfloat16* __restrict__ xin) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const float cv = vc[e];
+    const float vv = vu ? vu[e] + g * (cv - vu[e]) : cv;
+    const float xn = x[e] - dt * vv;
+    x[e] = xn;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(xn);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(xn - __bfloat162float(hi));
+    xin[(e >> 7) * 256 + (e & 127)] = hi;
+    xin[(e >> 7) * 256 + 128 + (e & 127)] = lo;
+  }
+}
+
+cudaError_t launch_euler_step(float* x, const float* vc, const float* vu, int64_t n, float dt, float guidance,
+                              __nv_bfloat16* xin, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  if (n & 127) return cudaErrorInvalidValue;
+  euler_step_kernel<<<grid_for(n), kThreads, 0, st>>>(x, vc, vu, n, dt, guidance, xin);
   return cudaGetLastError();
 }
 

@@ -78,6 +78,10 @@ cudaError_t launch_cfg_norm_partials(const float* vc, const float* vu, int64_t p
                                      double* part, cudaStream_t st);
 cudaError_t launch_euler_cfg_rescaled(float* x, const float* vc, const float* vu, int64_t per_sample, int B,
                                       float dt, float guidance, float phi, const double* part, __nv_bfloat16* xin,
-                                      cudaStream_t st);
+                                      int xin_copies, cudaStream_t st);
+// x -= dt (u + g (c - u)) (or dt c for vu == NULL) on n = rows x 128 values, with one
+// img_in operand row refreshed per token
+cudaError_t launch_euler_step(float* x, const float* vc, const float* vu, int64_t n, float dt, float guidance,
+                              __nv_bfloat16* xin, cudaStream_t st);
 
 }  // namespace lens

@@ -97,6 +97,16 @@ struct lens_dit {
     cudaGraphExec_t exec = nullptr;
     int64_t launches = 0;        // kernels one replay runs
   } sg;
+  // step-wise sampler (lens_sampler_prepare .. lens_sampler_finish); cleared by every
+  // call that reuses the modulation, text or token buffers
+  struct StepSampler {
+    bool ready = false;
+    int B = 0, gh = 0, gw = 0, n_txt = 0, steps = 0;
+    lens_sampler_options opt{};
+    bool masked = false;
+    TextLengths tl{};
+    double grid[kMaxTimesteps + 1];
+  } ss;
   // measurement
   int64_t launches = 0;
   int prof_kind = 0, prof_cap = 0, prof_n = 0;
@@ -727,7 +737,7 @@ static lens_status enqueue_sample(lens_dit* h, const uint16_t* txt_cond, const u
         const float* vu = h->vtok + (int64_t)B * per_sample;
         LENS_LAUNCH(h, 0, st, launch_cfg_norm_partials(h->vtok, vu, per_sample, B, guidance, h->cfgpart, st));
         LENS_LAUNCH(h, 0, st, launch_euler_cfg_rescaled(h->xtok, h->vtok, vu, per_sample, B, dt, guidance,
-                                                        o.cfg_rescale, h->cfgpart, h->xin, st));
+                                                        o.cfg_rescale, h->cfgpart, h->xin, 2, st));
       } else {
         LENS_LAUNCH(h, 0, st, launch_euler_cfg(h->xtok, h->vtok, per_sample, B, cfg, dt, guidance, h->xin, st));
       }
@@ -861,6 +871,7 @@ lens_status lens_dit_forward_masked(lens_dit* h, const float* img_tokens, int B,
                                     const uint16_t* txt, int n_txt, const int* txt_len, const float* t, float* v_out,
                                     void* stream) {
   if (!h || !img_tokens || !t || !v_out || (n_txt > 0 && !txt)) return LENS_ERR_INVALID_ARG;
+  h->ss.ready = false;
   TextLengths tl;
   if (txt_len) {
     if (B > kMaxRows) return LENS_ERR_SHAPE;
@@ -886,6 +897,7 @@ lens_status lens_dit_forward_masked(lens_dit* h, const float* img_tokens, int B,
 lens_status lens_dit_debug_blocks(lens_dit* h, int first, int last, float* h_img, float* h_txt, int B, int grid_h,
                                   int grid_w, int n_txt, const float* t, void* stream) {
   if (!h || !h_img || !t || (n_txt > 0 && !h_txt)) return LENS_ERR_INVALID_ARG;
+  h->ss.ready = false;
   lens_status s = check_sizes(h, B, grid_h, grid_w, n_txt);
   if (s) return s;
   if (B > h->cfg.max_timesteps) return LENS_ERR_SHAPE;
@@ -945,6 +957,7 @@ lens_status lens_sample_euler_ex(lens_dit* h, const uint16_t* txt_cond, const in
                                  int width_px, int steps, const lens_sampler_options* opt, uint64_t seed,
                                  float* latent_out, void* stream) {
   if (!h || !opt || !latent_out || (n_txt > 0 && !txt_cond)) return LENS_ERR_INVALID_ARG;
+  h->ss.ready = false;
   const float guidance = opt->guidance;
   if (steps < 1 || !isfinite(guidance)) return LENS_ERR_INVALID_ARG;
   if (!(opt->cfg_rescale >= 0.0f && opt->cfg_rescale <= 1.0f) || !isfinite(opt->shift_mu) ||
@@ -1069,6 +1082,7 @@ int64_t lens_dit_launch_count(lens_dit* h) { return h ? h->launches : 0; }
 lens_status lens_dit_op_timestep(lens_dit* h, const float* t, int T, float* temb, float* mod, void* stream) {
   if (!h || !t || (!temb && !mod)) return LENS_ERR_INVALID_ARG;
   if (T < 1 || T > h->cfg.max_timesteps) return LENS_ERR_SHAPE;
+  h->ss.ready = false;
   cudaStream_t st = (cudaStream_t)stream;
   lens_status s = compute_modulation(h, t, T, st);
   if (s) return s;
@@ -1080,6 +1094,7 @@ lens_status lens_dit_op_timestep(lens_dit* h, const float* t, int T, float* temb
 lens_status lens_dit_op_text_input(lens_dit* h, const uint16_t* txt, int B, int n_txt, float* c, void* stream) {
   if (!h || !txt || !c) return LENS_ERR_INVALID_ARG;
   if (B < 1 || n_txt < 1 || B > h->cfg.max_batch || n_txt > h->cfg.max_txt_tokens) return LENS_ERR_SHAPE;
+  h->ss.ready = false;
   cudaStream_t st = (cudaStream_t)stream;
   lens_status s = text_norm_rows(h, txt, B * n_txt, 0, st);
   if (s) return s;
@@ -1184,6 +1199,93 @@ lens_status lens_op_attention_masked(const uint16_t* q, const uint16_t* k, const
   return LENS_OK;
 }
 
+// ------------------------------------------------------------ step-wise sampler
+static lens_status check_options(const lens_sampler_options* o) {
+  if (!o || !isfinite(o->guidance)) return LENS_ERR_INVALID_ARG;
+  if (!(o->cfg_rescale >= 0.0f && o->cfg_rescale <= 1.0f) || !isfinite(o->shift_mu) || fabsf(o->shift_mu) > 50.0f)
+    return LENS_ERR_INVALID_ARG;
+  return LENS_OK;
+}
+
+lens_status lens_sampler_prepare(lens_dit* h, const uint16_t* txt, const int* txt_len, int B, int n_txt,
+                                 int height_px, int width_px, int steps, const lens_sampler_options* opt,
+                                 uint64_t seed, void* stream) {
+  if (!h) return LENS_ERR_INVALID_ARG;
+  h->ss.ready = false;
+  lens_status s = check_options(opt);
+  if (s) return s;
+  if (steps < 1) return LENS_ERR_INVALID_ARG;
+  if (height_px <= 0 || width_px <= 0 || height_px % 16 || width_px % 16) return LENS_ERR_SHAPE;
+  const int gh = height_px / 16, gw = width_px / 16, Ni = gh * gw;
+  if ((s = check_sizes(h, B, gh, gw, n_txt))) return s;
+  if (steps > h->cfg.max_timesteps) return LENS_ERR_SHAPE;
+  lens_dit::StepSampler& ss = h->ss;
+  ss.masked = txt_len != nullptr;
+  if (ss.masked) {
+    if (B > kMaxRows) return LENS_ERR_SHAPE;
+    for (int b = 0; b < B; ++b) {
+      if (txt_len[b] < 0 || txt_len[b] > n_txt) return LENS_ERR_SHAPE;
+      ss.tl.n[b] = txt_len[b];
+    }
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  sampler_time_grid(steps, opt->time_shift != 0, opt->shift_mu, ss.grid);
+  LENS_LAUNCH(h, 0, st, launch_noise_tokens(seed, B, gh, gw, h->xtok, st));
+  LENS_LAUNCH(h, 0, st, launch_tokens_to_operand(h->xtok, (int64_t)B * Ni, 1, (int64_t)B * Ni, h->xin, st));
+  if ((s = text_norm_rows(h, txt, B * n_txt, 0, st))) return s;     // NULL text: zeros
+  if ((s = text_in_gemm(h, B * n_txt, h->h_txt0, st))) return s;
+  float tv[kMaxTimesteps];
+  for (int k = 0; k < steps; ++k) tv[k] = (float)ss.grid[k];
+  if ((s = compute_modulation(h, tv, steps, st))) return s;
+  ss.B = B;
+  ss.gh = gh;
+  ss.gw = gw;
+  ss.n_txt = n_txt;
+  ss.steps = steps;
+  ss.opt = *opt;
+  ss.ready = true;
+  return LENS_OK;
+}
+
+lens_status lens_sampler_velocity(lens_dit* h, int k, float* v_out, void* stream) {
+  if (!h || !v_out || !h->ss.ready) return LENS_ERR_INVALID_ARG;
+  const lens_dit::StepSampler& ss = h->ss;
+  if (k < 0 || k >= ss.steps) return LENS_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(v_out) & 15) return LENS_ERR_INVALID_ARG;
+  return run_forward_core(h, ss.B, ss.gh, ss.gw, ss.n_txt, h->mod + (int64_t)k * h->modw, 0, v_out,
+                          ss.masked ? &ss.tl : nullptr, (cudaStream_t)stream);
+}
+
+lens_status lens_sampler_update(lens_dit* h, int k, const float* v_cond, const float* v_uncond, void* stream) {
+  if (!h || !v_cond || !h->ss.ready) return LENS_ERR_INVALID_ARG;
+  const lens_dit::StepSampler& ss = h->ss;
+  if (k < 0 || k >= ss.steps) return LENS_ERR_SHAPE;
+  const float g = ss.opt.guidance;
+  const bool cfg = g != 1.0f;
+  if (cfg && !v_uncond) return LENS_ERR_INVALID_ARG;
+  const bool shift = ss.opt.time_shift != 0;
+  const float dt = shift ? (float)(ss.grid[k] - ss.grid[k + 1]) : 1.0f / (float)ss.steps;
+  const int64_t per_sample = (int64_t)ss.gh * ss.gw * kInCh;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cfg && ss.opt.cfg_rescale != 0.0f) {
+    LENS_LAUNCH(h, 0, st, launch_cfg_norm_partials(v_cond, v_uncond, per_sample, ss.B, g, h->cfgpart, st));
+    LENS_LAUNCH(h, 0, st, launch_euler_cfg_rescaled(h->xtok, v_cond, v_uncond, per_sample, ss.B, dt, g,
+                                                    ss.opt.cfg_rescale, h->cfgpart, h->xin, 1, st));
+  } else {
+    LENS_LAUNCH(h, 0, st, launch_euler_step(h->xtok, v_cond, cfg ? v_uncond : nullptr, per_sample * ss.B, dt, g,
+                                            h->xin, st));
+  }
+  return LENS_OK;
+}
+
+lens_status lens_sampler_finish(lens_dit* h, float* latent_out, void* stream) {
+  if (!h || !latent_out || !h->ss.ready) return LENS_ERR_INVALID_ARG;
+  const lens_dit::StepSampler& ss = h->ss;
+  cudaStream_t st = (cudaStream_t)stream;
+  LENS_LAUNCH(h, 0, st, launch_unpatchify(h->xtok, ss.B, ss.gh, ss.gw, latent_out, st));
+  return LENS_OK;
+}
+
 lens_status lens_dit_op_euler_cfg_rescaled(lens_dit* h, float* x, const float* v_cond, const float* v_uncond, int B,
                                            int64_t per_sample, float dt, float guidance, float phi, void* stream) {
   if (!h || !x || !v_cond || !v_uncond) return LENS_ERR_INVALID_ARG;
@@ -1192,7 +1294,7 @@ lens_status lens_dit_op_euler_cfg_rescaled(lens_dit* h, float* x, const float* v
   cudaStream_t st = (cudaStream_t)stream;
   LENS_LAUNCH(h, 0, st, launch_cfg_norm_partials(v_cond, v_uncond, per_sample, B, guidance, h->cfgpart, st));
   LENS_LAUNCH(h, 0, st, launch_euler_cfg_rescaled(x, v_cond, v_uncond, per_sample, B, dt, guidance, phi, h->cfgpart,
-                                                  nullptr, st));
+                                                  nullptr, 1, st));
   return LENS_OK;
 }
 

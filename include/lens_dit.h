@@ -210,6 +210,37 @@ LENS_API lens_status lens_sample_euler_ex(lens_dit* h, const uint16_t* txt_cond,
                                           int height_px, int width_px, int steps, const lens_sampler_options* opt,
                                           uint64_t seed, float* latent_out, void* stream);
 
+/* Step-wise sampler: the pieces of lens_sample_euler_ex as separate calls, for a
+ * caller that evaluates the conditional and the unconditional half of CFG in two
+ * processes (one per GPU) and exchanges the two velocities between steps.  The
+ * velocity of one batch row does not depend on the other rows, so two handles
+ * running the halves and exchanging velocities reproduce lens_sample_euler_ex.
+ * Summary page "Lens: 重新思考基础文生图模型的训练效率", "方法步骤详情" (20 steps,
+ * CFG 5.0) and blog "Lens", "Exploring Image Editing" (uncond + s (cond - uncond)):
+ * each step needs both halves once.
+ *
+ * lens_sampler_prepare: seeded noise x (as lens_sample_euler), the text input of
+ *   `txt` (dev bf16 [B, n_txt, 4, 2880]; NULL = zeros, the unconditional text of the
+ *   plain sampler) with optional lengths txt_len (host int [B], NULL = all valid),
+ *   and the modulation of every step (steps <= max_timesteps).  The state lives in
+ *   the handle until the next call that is not one of these four.
+ * lens_sampler_velocity: the velocity of this handle's rows at step k (0-based),
+ *   v_out dev fp32 [B, (height/16)*(width/16), 128], 16-byte aligned.
+ * lens_sampler_update: x -= dt_k v with v = v_cond when opt.guidance == 1, else the
+ *   plain or norm-rescaled combination of v_cond and v_uncond (both dev fp32, same
+ *   layout as v_out; v_uncond ignored when guidance == 1).
+ * lens_sampler_finish: latent_out dev fp32 [B, 32, height/8, width/8] from x.
+ * Errors: INVALID_ARG (NULL, bad options as lens_sample_euler_ex, steps < 1, a step
+ * call without a prepared state, unaligned v_out), SHAPE (sizes as
+ * lens_sample_euler, steps > max_timesteps, k outside [0, steps)). */
+LENS_API lens_status lens_sampler_prepare(lens_dit* h, const uint16_t* txt, const int* txt_len, int B, int n_txt,
+                                          int height_px, int width_px, int steps, const lens_sampler_options* opt,
+                                          uint64_t seed, void* stream);
+LENS_API lens_status lens_sampler_velocity(lens_dit* h, int k, float* v_out, void* stream);
+LENS_API lens_status lens_sampler_update(lens_dit* h, int k, const float* v_cond, const float* v_uncond,
+                                         void* stream);
+LENS_API lens_status lens_sampler_finish(lens_dit* h, float* latent_out, void* stream);
+
 /* Test hook: run blocks [first, last) in place on a residual stream.
  *   h_img dev fp32 [B, grid_h*grid_w, 1536], h_txt dev fp32 [B, n_txt, 1536]
  *   t host fp32 [B].  Errors as lens_dit_forward, plus SHAPE for a bad range. */

@@ -365,3 +365,60 @@ def test_sampler_options_are_part_of_the_replay_key(small):
             L.lens_sample_euler_ex(h, E, None, None, None, B, nt, 16 * gh, 16 * gw, 3, opt, 5, out)
             L.lens_dit_sync(h, s)
             assert np.array_equal(host(out), refs[want])
+
+
+# ------------------------------------------------------------------ step-wise sampler / CFG split
+@pytest.mark.parametrize("gh,gw,nt,steps,phi,mu", [(8, 6, 16, 3, 0.0, None), (64, 64, 256, 2, 1.0, 0.8)])
+def test_cfg_split_halves_reproduce_the_fused_sampler(small, gh, gw, nt, steps, phi, mu):
+    """Two handles stand in for the two ranks of a CFG pair (one GPU: run in turn,
+    the exchange is a shared buffer).  Both end on the fused sampler's latent, bit
+    for bit: a batch row's velocity does not depend on the other rows."""
+    d, w, h = small
+    h2 = _handle(w, 2, max_batch=4, max_img=8192, max_txt=256)
+    try:
+        B, seed = 1, 7
+        Ec = dev(text_features(B, nt, 61))
+        opt = _options(5.0, phi, mu)
+        shape = (B, 32, 2 * gh, 2 * gw)
+        ref = torch.empty(shape, dtype=torch.float32, device="cuda")
+        L.lens_sample_euler_ex(h, Ec, None, None, None, B, nt, 16 * gh, 16 * gw, steps, opt, seed, ref)
+        _sync(h)
+        L.lens_sampler_prepare(h, Ec, None, B, nt, 16 * gh, 16 * gw, steps, opt, seed)
+        L.lens_sampler_prepare(h2, None, None, B, nt, 16 * gh, 16 * gw, steps, opt, seed)
+        v_all = torch.empty((2, B, gh * gw, 128), dtype=torch.float32, device="cuda")
+        for k in range(steps):
+            L.lens_sampler_velocity(h, k, v_all[0])
+            L.lens_sampler_velocity(h2, k, v_all[1])
+            L.lens_sampler_update(h, k, v_all[0], v_all[1])
+            L.lens_sampler_update(h2, k, v_all[0], v_all[1])
+        outs = [torch.empty(shape, dtype=torch.float32, device="cuda") for _ in range(2)]
+        L.lens_sampler_finish(h, outs[0])
+        L.lens_sampler_finish(h2, outs[1])
+        _sync(h)
+        assert np.array_equal(host(outs[0]), host(outs[1]))
+        assert np.array_equal(host(outs[0]), host(ref))
+    finally:
+        h2.destroy()
+
+
+def test_step_sampler_state_rules(small):
+    d, w, h = small
+    B, gh, gw, nt = 1, 4, 4, 16
+    Ec = dev(text_features(B, nt, 62))
+    opt = _options(1.0, 0.0, None)
+    v = torch.empty((B, gh * gw, 128), dtype=torch.float32, device="cuda")
+    L.lens_sampler_prepare(h, Ec, None, B, nt, 16 * gh, 16 * gw, 2, opt, 3)
+    L.lens_sampler_velocity(h, 1, v)
+    with pytest.raises(L.LensError) as e:
+        L.lens_sampler_velocity(h, 2, v)                       # k past the last step
+    assert e.value.status == 2
+    with pytest.raises(L.LensError) as e:
+        L.lens_sampler_prepare(h, Ec, None, B, nt, 16 * gh, 16 * gw, 65, opt, 3)   # > max_timesteps
+    assert e.value.status == 2
+    L.lens_sampler_prepare(h, Ec, None, B, nt, 16 * gh, 16 * gw, 2, opt, 3)
+    X = dev(np.zeros((B, gh * gw, 128), np.float32))
+    L.lens_dit_forward(h, X, B, gh, gw, Ec, nt, [0.5], v)       # reuses the buffers: state dropped
+    with pytest.raises(L.LensError) as e:
+        L.lens_sampler_update(h, 0, v, None)
+    assert e.value.status == 1
+    _sync(h)
