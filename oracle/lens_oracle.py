@@ -19,7 +19,8 @@ Sources (page title, section):
             "自适应调制与 RMSNorm", "3D RoPE 旋转位置编码", "多层级文本特征融合",
             "Patchify 补丁化与输出投影", "guidance 1.0".
   [int4]    "从提示词到成图：Lens-3.8B-4bit完整管线解析", section 4 (DiT: 128-channel input,
-            patch 2, 32-channel output, time_text_embed, axes [8, 28, 28]) and section 6
+            patch 2, 32-channel output, time_text_embed, axes [8, 28, 28]; int4 weights with
+            group_size 64, sensitive layers in bf16, about 2.35 GB) and section 6
             (pipeline call with steps and seed).
   [survey]  "SOTA image generation" survey page, sections "CFG：无分类器引导" and
             "交叉注意力与条件注入" (joint attention over the concatenated sequence).
@@ -456,6 +457,75 @@ def sample(W: Weights, dims, E_cond: np.ndarray, E_uncond: Optional[np.ndarray],
                 cfg_rescaled(vv[:B], vv[B:], guidance, phi)
         x = euler(x, unpatchify(v, grid_h, grid_w, C, p), dt)
     return x
+
+
+# ============================================================ int4 weight-only (4-bit page)
+W4_GROUP = 64
+W4_SENSITIVE = ("img_in", "txt_in", "proj_out", "time_text_embed", "norm_out")
+
+
+def _bf16_rne(x: np.ndarray) -> np.ndarray:
+    """fp32 -> nearest bf16 (ties to even), returned as fp32 (finite inputs)."""
+    u = np.asarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32)
+
+
+def w4_quantizable(name: str, ndim: int) -> bool:
+    """[int4] section 4: the DiT stores its weights in 4 bits with group_size 64 and
+    keeps img_in, txt_in, proj_out, time_text_embed and norm_out in bf16.  READING:
+    every other Linear weight (all 2-D weights inside the 48 blocks: qkv, to_out,
+    to_add_out, w1/w2/w3, img_mod/txt_mod) is quantized; gains and biases are not."""
+    return ndim == 2 and name.endswith(".weight") and not name.startswith(W4_SENSITIVE)
+
+
+def quantize_w4(w: np.ndarray, group: int = W4_GROUP):
+    """Affine 4-bit quantization of a [N, K] weight in groups of `group` along K.
+    [int4] section 4 gives the bit width and the group size only.  READING: per group
+    scale s = (max - min) / 15 and bias b = min, both stored as bf16 (16 bits each:
+    with 4-bit codes this is the 2.35 GB the page gives for the whole model), codes
+    q = clamp(rint((w - b) / s), 0, 15) computed in fp32 with the stored s and b
+    (q = 0 where s = 0).  w is fp32 (or bf16 bits).  Returns (q uint8 [N, K],
+    s fp32 [N, K/group], b fp32 [N, K/group]); s and b hold bf16 values."""
+    w = upcast(w, np.float32)
+    N, K = w.shape
+    if K % group:
+        raise ValueError(f"K = {K} is not a multiple of the group size {group}")
+    g = w.reshape(N, K // group, group)
+    mn, mx = g.min(axis=-1), g.max(axis=-1)
+    sc = _bf16_rne((mx - mn) / np.float32(15.0))
+    bi = _bf16_rne(mn)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.rint((g - bi[..., None]) / sc[..., None])
+    q = np.where(sc[..., None] > 0, q, 0.0)
+    q = np.clip(q, 0, 15).astype(np.uint8).reshape(N, K)
+    return q, sc, bi
+
+
+def dequantize_w4(q: np.ndarray, sc: np.ndarray, bi: np.ndarray, group: int = W4_GROUP) -> np.ndarray:
+    """w' = s q + b per group, exactly (fp64)."""
+    N, K = q.shape
+    g = q.reshape(N, K // group, group).astype(F64)
+    return (g * sc.astype(F64)[..., None] + bi.astype(F64)[..., None]).reshape(N, K)
+
+
+def quantize_model_w4(tensors: Mapping[str, np.ndarray]) -> Dict[str, np.ndarray]:
+    """The model the 4-bit pipeline evaluates: quantizable weights replaced by their
+    dequantized values (fp64), everything else unchanged (bf16 bits)."""
+    out = {}
+    for name, w in tensors.items():
+        out[name] = dequantize_w4(*quantize_w4(w)) if w4_quantizable(name, np.ndim(w)) else w
+    return out
+
+
+def w4_model_bytes(tensors_or_shapes) -> int:
+    """Stored bytes of the 4-bit model: 4-bit codes plus a bf16 scale and a bf16 bias
+    per group for quantizable weights, 2 bytes per value for the rest."""
+    total = 0
+    for name, shape in tensors_or_shapes:
+        n = int(np.prod(shape))
+        total += n // 2 + (n // W4_GROUP) * 4 if w4_quantizable(name, len(shape)) else 2 * n
+    return total
 
 
 # ============================================================ model size

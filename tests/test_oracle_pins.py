@@ -402,6 +402,68 @@ def test_cfg_rescaled_values_and_invariants():
     assert np.allclose(o.sample_euler(vel, np.zeros(4), 2, 5.0, phi=1.0), 1.0, atol=1e-15)
 
 
+# ------------------------------------------------------------------ int4 weight-only
+def test_w4_model_size_matches_the_page():
+    g = {k: v for k, v in _golden("lens_int4_model.txt")}
+    assert int(g["bits"]) == 4 and int(g["group_size"]) == o.W4_GROUP
+    specs = [(n, s) for n, s, _ in weight_specs(LENS)]
+    gb = o.w4_model_bytes(specs) / 1e9
+    assert abs(gb - float(g["model_GB"])) < 0.01, gb          # 2.349 GB
+    # the sensitive layers stay bf16, every 2-D block weight is quantized
+    for name, shape in specs:
+        q = o.w4_quantizable(name, len(shape))
+        assert q == (len(shape) == 2 and name.startswith("transformer_blocks.")), name
+
+
+def test_w4_hand_worked_groups():
+    # codes 0..15 spread over a group: min 0, max 15 -> s = 1, b = 0, q = w, exact
+    w = np.tile(np.arange(16, dtype=np.float32), 8).reshape(2, 64)
+    q, sc, bi = o.quantize_w4(w)
+    assert np.array_equal(q, w.astype(np.uint8)) and np.all(sc == 1.0) and np.all(bi == 0.0)
+    assert np.array_equal(o.dequantize_w4(q, sc, bi), w)
+    # a shifted, scaled copy: w = 0.5 + 0.25 k -> s = 0.25, b = 0.5, same codes
+    q2, sc2, bi2 = o.quantize_w4(0.5 + 0.25 * w)
+    assert np.array_equal(q2, q) and np.all(sc2 == 0.25) and np.all(bi2 == 0.5)
+    # a constant group: s = 0, every code 0, the value comes back as its bf16 bias
+    c = np.full((1, 64), 0.375, np.float32)
+    q3, sc3, bi3 = o.quantize_w4(c)
+    assert np.all(q3 == 0) and sc3[0, 0] == 0.0 and np.array_equal(o.dequantize_w4(q3, sc3, bi3), c)
+    # rint ties go to even: 1.5 -> 2, 2.5 -> 2 (group min 0, max 15)
+    t = np.zeros((1, 64), np.float32)
+    t[0, 1], t[0, 2], t[0, 3] = 15.0, 1.5, 2.5
+    assert o.quantize_w4(t)[0][0, 2] == 2 and o.quantize_w4(t)[0][0, 3] == 2
+
+
+def test_w4_error_bound_and_order_on_random_weights():
+    rng = np.random.default_rng(14)
+    w = (rng.standard_normal((96, 1536)) * 0.02).astype(np.float32)
+    q, sc, bi = o.quantize_w4(w)
+    assert q.dtype == np.uint8 and q.max() <= 15 and sc.shape == (96, 24)
+    err = np.abs(o.dequantize_w4(q, sc, bi) - w).reshape(96, 24, 64)
+    g = w.reshape(96, 24, 64)
+    # half a step, plus what rounding the bias to bf16 moved the grid
+    bound = 0.5 * sc + np.abs(g.min(-1) - bi) + 1e-9
+    assert np.all(err.max(-1) <= bound[...] + 0.5 * sc * 2.0 ** -7)
+    # codes keep the order of the values inside a group
+    order = np.argsort(g, axis=-1, kind="stable")
+    qs = np.take_along_axis(q.reshape(96, 24, 64), order, -1)
+    assert np.all(np.diff(qs.astype(int), axis=-1) >= 0)
+    # the extremes of a group land on codes 0 and 15 (or one step inside)
+    assert np.all(np.take_along_axis(q.reshape(96, 24, 64), order[..., :1], -1) <= 1)
+    assert np.all(np.take_along_axis(q.reshape(96, 24, 64), order[..., -1:], -1) >= 14)
+
+
+def test_w4_model_replaces_only_quantizable_weights():
+    import dataclasses
+    w = make_weights(dataclasses.replace(TINY, mlp_hidden=128), seed=3)      # every K a multiple of 64
+    qm = o.quantize_model_w4(w)
+    for name, t in w.items():
+        if o.w4_quantizable(name, t.ndim):
+            assert qm[name].dtype == np.float64 and not np.array_equal(qm[name], o.upcast(t))
+        else:
+            assert qm[name] is t
+
+
 # ------------------------------------------------------------------ noise
 def test_splitmix64_published_vectors():
     want = [int(r[0], 16) for r in _golden("splitmix64_seed0.txt")]
