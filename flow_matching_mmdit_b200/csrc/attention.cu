@@ -57,7 +57,10 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 //               exponentials run, and the two tiles ping-pong on the tensor cores
 //   warp 8      TMA: both Q tiles once, then K and V tiles of 128 keys (3 stages)
 //   warp 9      UMMA issuer: S_X = Q_X K_j^T (M=128, N=128, K=64) and
-//               O_X += P_X V_j (M=128, N=64, K=128) with P_X read from TMEM
+//               O_X += P_X V_j (M=128, N=64, K=128) with P_X read from TMEM.
+//               A wait in this thread stalls until its queued UMMAs are accepted,
+//               so the waits S_0 and S_1 need (K/V stage, both S slots released)
+//               are taken back to back: the queue drains once for them.
 // The running max m and sum l of each row live in registers; O_X is rescaled in
 // TMEM only when m grows by more than 2^8 (softmax is invariant to the subtracted
 // constant, so a stale max is exact up to rounding).
@@ -171,23 +174,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int j = 0; ok && j <= nkv; ++j) {
         if (j < nkv) {
           const int s = j % STAGES;
-          if (!mbar_wait(&bar.kv_full[s], (j / STAGES) & 1, err)) break;
+          // every wait S_0[j] and S_1[j] need, back to back: only the first drains the queue
+          ok = mbar_wait(&bar.kv_full[s], (j / STAGES) & 1, err) &&
+               (j == 0 || (mbar_wait(&bar.s_free[0], (j - 1) & 1, err) && mbar_wait(&bar.s_free[1], (j - 1) & 1, err)));
+          if (!ok) break;
           tc_fence_after();
           const uint64_t kdesc = umma_desc_sw128(smem_u32(sKV + s * 2 * KV_BYTES));
 #pragma unroll
           for (int x = 0; x < TILES; ++x) {
-            if (j > 0 && !mbar_wait(&bar.s_free[x], (j - 1) & 1, err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
             const uint64_t qdesc = umma_desc_sw128(smem_u32(sQ + x * Q_BYTES));
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               umma_bf16(tmem + x * 128, qdesc + 2 * k, kdesc + 2 * k, idesc_s, k > 0 ? 1u : 0u);
             umma_commit(&bar.s_full[x]);
           }
-          if (!ok) break;
         }
         if (j >= 1) {
           const int jj = j - 1;
