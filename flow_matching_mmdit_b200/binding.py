@@ -28,7 +28,7 @@ EXPORTS = [
     "lens_op_timestep_embed_noalloc", "lens_dit_forward_masked", "lens_sample_euler_masked",
     "lens_op_attention_masked", "lens_sampler_default_options", "lens_shift_mu", "lens_time_grid",
     "lens_sample_euler_ex", "lens_dit_op_euler_cfg_rescaled", "lens_sampler_prepare", "lens_sampler_velocity",
-    "lens_sampler_update", "lens_sampler_finish",
+    "lens_sampler_update", "lens_sampler_finish", "lens_op_quantize_w4", "lens_op_gemm_w4",
 ]
 
 KERNELS = {"none": 0, "attention": 1, "gemm_qkv": 2, "gemm_out": 3, "gemm_w13": 4, "gemm_w2": 5, "rmsnorm_mod": 6,
@@ -47,7 +47,8 @@ class lens_dit_config(ctypes.Structure):
                 ("latent_channels", ctypes.c_int), ("patch", ctypes.c_int), ("txt_layers", ctypes.c_int),
                 ("txt_dim", ctypes.c_int), ("rope_axes", ctypes.c_int * 3), ("rope_theta", ctypes.c_float),
                 ("eps", ctypes.c_float), ("freq_dim", ctypes.c_int), ("max_batch", ctypes.c_int),
-                ("max_img_tokens", ctypes.c_int), ("max_txt_tokens", ctypes.c_int), ("max_timesteps", ctypes.c_int)]
+                ("max_img_tokens", ctypes.c_int), ("max_txt_tokens", ctypes.c_int), ("max_timesteps", ctypes.c_int),
+                ("weight_bits", ctypes.c_int)]
 
 
 class lens_sampler_options(ctypes.Structure):
@@ -110,6 +111,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lens_sampler_velocity": (I, [P, I, P, P]),
         "lens_sampler_update": (I, [P, I, P, P, P]),
         "lens_sampler_finish": (I, [P, P, P]),
+        "lens_op_quantize_w4": (I, [P, L, L, P, P, P]),
+        "lens_op_gemm_w4": (I, [P, P, P, P, P, I, I, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -353,6 +356,16 @@ def lens_op_attention_masked(q, k, v, B: int, n_txt: int, n_img: int, txt_len, o
     _check(load_library().lens_op_attention_masked(_ptr(q), _ptr(k), _ptr(v), B, n_txt, n_img, _iptr(ln),
                                                    _ptr(out_txt), _ptr(out_img), _stream(stream)),
            "lens_op_attention_masked")
+
+
+def lens_op_quantize_w4(w, rows: int, k: int, codes, scales, stream=None) -> None:
+    _check(load_library().lens_op_quantize_w4(_ptr(w), rows, k, _ptr(codes), _ptr(scales), _stream(stream)),
+           "lens_op_quantize_w4")
+
+
+def lens_op_gemm_w4(A, codes, scales, bias, C, M: int, N: int, K: int, stream=None) -> None:
+    _check(load_library().lens_op_gemm_w4(_ptr(A), _ptr(codes), _ptr(scales), _ptr(bias), _ptr(C), M, N, K,
+                                          _stream(stream)), "lens_op_gemm_w4")
 
 
 def lens_op_euler_cfg(x, v_cond, v_uncond, n: int, dt: float, guidance: float, stream=None) -> None:

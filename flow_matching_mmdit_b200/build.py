@@ -21,7 +21,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "liblens_dit.so")
 INCLUDE = os.path.join(ROOT, "include")
 
-SOURCES = ["lens_dit.cu", "gemm.cu", "attention.cu", "elementwise.cu", "noalloc.cu"]
+SOURCES = ["lens_dit.cu", "gemm.cu", "attention.cu", "elementwise.cu", "noalloc.cu", "w4.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -104,6 +104,33 @@ bool encode_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_tmap_w4_codes(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t k, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || k == 0 || k % 64 || box_rows == 0 || box_rows > 256) return false;
+  if (reinterpret_cast<uintptr_t>(ptr) & 15) return false;
+  const cuuint64_t dims[2] = {k / 2, rows};
+  const cuuint64_t strides[1] = {k / 2};
+  const cuuint32_t box[2] = {32, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_tmap_w4_scales(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t k, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows == 0 || rows % 4 || k == 0 || k % 64 || box_rows == 0 || box_rows > 256 || box_rows % 4)
+    return false;
+  if (reinterpret_cast<uintptr_t>(ptr) & 15) return false;
+  const cuuint64_t dims[2] = {rows, k / 64};
+  const cuuint64_t strides[1] = {rows * 4};
+  const cuuint32_t box[2] = {box_rows, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 void finalize_problems(GemmArgs& a, int bn, int bm) {
   int begin = 0;
   for (int i = 0; i < a.num_problems; ++i) {

@@ -22,6 +22,36 @@ bool encode_tmap_out(CUtensorMap* m, const void* ptr, int elem_bytes, uint64_t r
 // box = d0 x box_rows x 1, 128-byte swizzle, zero fill out of bounds.
 bool encode_tmap_bf16_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box_rows);
 
+// 4-bit weights (int4 weight-only path, w4.cu).  A quantized [rows, k] matrix is
+//   codes  uint8 [rows, k / 2]: 32-bit word w of a row holds the codes of k in
+//          [8w, 8w + 8); the code of k = 8w + 2j sits in bits [4j, 4j + 4), that of
+//          k = 8w + 2j + 1 in bits [16 + 4j, 20 + 4j) (j = 0..3), so one shift and
+//          mask gives the bf16 pair (128 + q_2j, 128 + q_2j+1) after an OR with 0x43004300
+//   scales uint32 [k / 64, rows]: group g of row r at [g][r], bf16 scale in the low
+//          half, bf16 bias in the high half; w = scale * q + bias
+// codes map: box 32 bytes (one 64-wide k block) x box_rows rows, no swizzle;
+// scales map: box box_rows x 1 group (box_rows a multiple of 4).
+bool encode_tmap_w4_codes(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t k, uint32_t box_rows);
+bool encode_tmap_w4_scales(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t k, uint32_t box_rows);
+
+// Quantize bf16 w [rows, k] (k a multiple of 64) into the layout above: per group of
+// 64 along k, scale = bf16((max - min) / 15), bias = bf16(min), code =
+// clamp(rint((w - bias) / scale), 0, 15) in fp32 (0 where scale = 0).  The scales of
+// group g, row r go to scales[g * scale_ld + r] (scale_ld >= rows: the rows of a
+// larger matrix this one is a row slice of, with scales pre-offset by its first row).
+cudaError_t launch_quantize_w4(const void* w_bf16, int64_t rows, int64_t k, uint8_t* codes, uint32_t* scales,
+                               int64_t scale_ld, cudaStream_t st);
+
+// GEMM with one 4-bit operand, dequantized in shared memory.  quant_a = false: B
+// (the N side, weights [N, K]) is 4-bit, A0/A1 are bf16 maps as for launch_gemm;
+// quant_a = true: A (the M side, weights of the swap-AB modulation GEMM) is 4-bit
+// and B0 is a bf16 map.  Q*/S* are the codes / scales maps (box rows = bn for B,
+// 128 for A).  Same problems, epilogues and output maps as launch_gemm.
+cudaError_t launch_gemm_w4(int bn, int epi, bool quant_a, const CUtensorMap* A0, const CUtensorMap* B0,
+                           const CUtensorMap* Q0, const CUtensorMap* S0, const CUtensorMap* A1, const CUtensorMap* B1,
+                           const CUtensorMap* Q1, const CUtensorMap* S1, const CUtensorMap* C0, const CUtensorMap* C1,
+                           GemmArgs& args, int sms, cudaStream_t st);
+
 // Fill tile counts of args.p[0..num_problems) for tile width bn and launch the
 // persistent kernel (grid = min(tiles, sms)).  (bn, epi) must be an instantiated pair.
 // C0 / C1 are the output maps of the TMA-store epilogues (EPI_F32, EPI_RESID,

@@ -20,11 +20,22 @@ using namespace lens;
 
 namespace {
 
+// the largest block weight staged at create with weight_bits = 4 (one stream's AdaLN)
+constexpr size_t kStageElems = (size_t)kModPerStream * kHidden;
+
 constexpr int kBnQkv = 192, kBnOut = 192, kBnW13 = 256, kBnW2 = 192, kBnImgIn = 256, kBnTxtIn = 128,
               kBnProj = 128;
 
+// a 4-bit weight (weight_bits = 4): codes and scales in lens_op_quantize_w4's layout
+struct QW {
+  uint8_t* codes = nullptr;
+  uint32_t* scales = nullptr;
+  CUtensorMap tq, ts;
+};
+
 struct StreamW {
-  __nv_bfloat16 *qkv, *out, *w13, *w2;
+  __nv_bfloat16 *qkv, *out, *w13, *w2;   // bf16 weights (null with weight_bits = 4)
+  QW q_qkv, q_out, q_w13, q_w2;          // 4-bit weights (weight_bits = 4)
   float *b_qkv, *b_out, *b_w13, *b_w2, *gq, *gk;
   CUtensorMap t_qkv, t_out, t_w13, t_w2;
   // a bias that is absent or all zero is not added at all
@@ -73,6 +84,12 @@ struct lens_dit {
   float *b_t1, *b_t2, *b_txt_in, *b_img_in, *b_proj, *b_mod, *g_txt;
   bool has_b_txt_in = false, has_b_img_in = false, has_b_proj = false;
   CUtensorMap t_txt_in, t_img_in, t_proj, t_mod;
+  // weight_bits = 4: block AdaLN rows as 4-bit, norm_out rows in bf16 (w_no)
+  bool w4 = false;
+  QW q_mod;
+  __nv_bfloat16* w_no = nullptr;
+  CUtensorMap t_no;
+  __nv_bfloat16* wstage = nullptr;      // create-time staging of one bf16 matrix
   std::vector<BlockW> blk;
   // workspace
   void* ws = nullptr;
@@ -235,7 +252,15 @@ static void layout_weights(lens_dit* h, Bump& b) {
   h->w_txt_in = b.take<__nv_bfloat16>((size_t)kHidden * kTxtLayers * kTxtDim);
   h->w_img_in = b.take<__nv_bfloat16>((size_t)kHidden * 2 * kInCh);
   h->w_proj = b.take<__nv_bfloat16>((size_t)kInCh * kHidden);
-  h->w_mod = b.take<__nv_bfloat16>((size_t)h->modw * kHidden);
+  if (h->w4) {
+    const size_t mrows = (size_t)nb * kModPerBlock;
+    h->w_mod = nullptr;
+    h->w_no = b.take<__nv_bfloat16>((size_t)2 * kHidden * kHidden);
+    h->q_mod.codes = b.take<uint8_t>(mrows * kHidden / 2);
+    h->q_mod.scales = b.take<uint32_t>(mrows * (kHidden / 64));
+  } else {
+    h->w_mod = b.take<__nv_bfloat16>((size_t)h->modw * kHidden);
+  }
   h->b_t1 = b.take<float>(kHidden);
   h->b_t2 = b.take<float>(kHidden);
   h->b_txt_in = b.take<float>(kHidden);
@@ -247,10 +272,22 @@ static void layout_weights(lens_dit* h, Bump& b) {
   for (int i = 0; i < nb; ++i)
     for (int s = 0; s < 2; ++s) {
       StreamW& w = h->blk[i].s[s];
-      w.qkv = b.take<__nv_bfloat16>((size_t)3 * kHidden * kHidden);
-      w.out = b.take<__nv_bfloat16>((size_t)kHidden * kHidden);
-      w.w13 = b.take<__nv_bfloat16>((size_t)2 * kMlp * kHidden);
-      w.w2 = b.take<__nv_bfloat16>((size_t)kHidden * kMlp);
+      if (h->w4) {
+        auto take_q = [&b](QW& q, size_t rows, size_t k) {
+          q.codes = b.take<uint8_t>(rows * k / 2);
+          q.scales = b.take<uint32_t>(rows * (k / 64));
+        };
+        w.qkv = w.out = w.w13 = w.w2 = nullptr;
+        take_q(w.q_qkv, 3 * kHidden, kHidden);
+        take_q(w.q_out, kHidden, kHidden);
+        take_q(w.q_w13, 2 * kMlp, kHidden);
+        take_q(w.q_w2, kHidden, kMlp);
+      } else {
+        w.qkv = b.take<__nv_bfloat16>((size_t)3 * kHidden * kHidden);
+        w.out = b.take<__nv_bfloat16>((size_t)kHidden * kHidden);
+        w.w13 = b.take<__nv_bfloat16>((size_t)2 * kMlp * kHidden);
+        w.w2 = b.take<__nv_bfloat16>((size_t)kHidden * kMlp);
+      }
       w.b_qkv = b.take<float>(3 * kHidden);
       w.b_out = b.take<float>(kHidden);
       w.b_w13 = b.take<float>(2 * kMlp);
@@ -258,6 +295,20 @@ static void layout_weights(lens_dit* h, Bump& b) {
       w.gq = b.take<float>(kHeadDim);
       w.gk = b.take<float>(kHeadDim);
     }
+}
+
+// A block Linear weight [rows, k]: bf16 straight copy, or (weight_bits = 4) staged
+// on the device and quantized into q at row offset row0 of a matrix of scale_ld rows.
+static lens_status put_block_weight(lens_dit* h, __nv_bfloat16* dst, QW* q, const uint16_t* src, size_t rows,
+                                    size_t k, size_t row0 = 0, size_t scale_ld = 0) {
+  if (!h->w4) return put_bf16(dst, src, rows * k);
+  if (!h->wstage || rows * k > kStageElems) return LENS_ERR_CUDA;
+  if (cudaMemcpy(h->wstage, src, rows * k * 2, cudaMemcpyHostToDevice) != cudaSuccess) return LENS_ERR_CUDA;
+  if (launch_quantize_w4(h->wstage, (int64_t)rows, (int64_t)k, q->codes + row0 * k / 2, q->scales + row0,
+                         (int64_t)(scale_ld ? scale_ld : rows), nullptr) != cudaSuccess)
+    return LENS_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return LENS_ERR_CUDA;   // wstage is reused by the next weight
+  return LENS_OK;
 }
 
 static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
@@ -342,7 +393,7 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
   // all AdaLN projections: block-major, image then text, then norm_out
   const int64_t no_off = (int64_t)nb * kModPerBlock;
   if (!(w = L.get("norm_out.linear.weight", {2 * D, D}, true))) return L.st;
-  if ((st = put_bf16(h->w_mod + no_off * D, w, (size_t)2 * D * D))) return st;
+  if ((st = put_bf16(h->w4 ? h->w_no : h->w_mod + no_off * D, w, (size_t)2 * D * D))) return st;
   if ((st = put_f32(h->b_mod + no_off, L.get("norm_out.linear.bias", {2 * D}, false), 2 * D, 0.f, stage)))
     return st;
 
@@ -353,13 +404,15 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
       const std::string mod = p + (s == 0 ? "img_mod" : "txt_mod");
       const int64_t moff = (int64_t)i * kModPerBlock + s * kModPerStream;
       if (!(w = L.get(mod + ".weight", {kModPerStream, D}, true))) return L.st;
-      if ((st = put_bf16(h->w_mod + moff * D, w, (size_t)kModPerStream * D))) return st;
+      if ((st = put_block_weight(h, h->w4 ? nullptr : h->w_mod + moff * D, &h->q_mod, w, kModPerStream, D, moff,
+                                 (size_t)nb * kModPerBlock)))
+        return st;
       if ((st = put_f32(h->b_mod + moff, L.get(mod + ".bias", {kModPerStream}, false), kModPerStream, 0.f, stage)))
         return st;
 
       const std::string qkv = p + (s == 0 ? "attn.img_qkv" : "attn.txt_qkv");
       if (!(w = L.get(qkv + ".weight", {3 * D, D}, true))) return L.st;
-      if ((st = put_bf16(sw.qkv, w, (size_t)3 * D * D))) return st;
+      if ((st = put_block_weight(h, sw.qkv, &sw.q_qkv, w, 3 * D, D))) return st;
       sw.has_b_qkv = any_nonzero_bf16(L.get(qkv + ".bias", {3 * D}, false), 3 * D);
       if ((st = put_f32(sw.b_qkv, L.get(qkv + ".bias", {3 * D}, false), 3 * D, 0.f, stage))) return st;
       const std::string nq = p + (s == 0 ? "attn.norm_q" : "attn.norm_added_q");
@@ -372,7 +425,7 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
 
       const std::string out = p + (s == 0 ? "attn.to_out" : "attn.to_add_out");
       if (!(w = L.get(out + ".weight", {D, D}, true))) return L.st;
-      if ((st = put_bf16(sw.out, w, (size_t)D * D))) return st;
+      if ((st = put_block_weight(h, sw.out, &sw.q_out, w, D, D))) return st;
       sw.has_b_out = any_nonzero_bf16(L.get(out + ".bias", {D}, false), D);
       if ((st = put_f32(sw.b_out, L.get(out + ".bias", {D}, false), D, 0.f, stage))) return st;
 
@@ -388,7 +441,7 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
         memcpy(&pack[(size_t)(64 * c) * D], w1 + (size_t)(32 * c) * D, (size_t)32 * D * 2);
         memcpy(&pack[(size_t)(64 * c + 32) * D], w3 + (size_t)(32 * c) * D, (size_t)32 * D * 2);
       }
-      if ((st = put_bf16(sw.w13, pack.data(), pack.size()))) return st;
+      if ((st = put_block_weight(h, sw.w13, &sw.q_w13, pack.data(), 2 * kMlp, D))) return st;
       const uint16_t* b1 = L.get(mlp + ".w1.bias", {kMlp}, false);
       const uint16_t* b3 = L.get(mlp + ".w3.bias", {kMlp}, false);
       if (L.st) return L.st;
@@ -401,7 +454,7 @@ static lens_status load_weights(lens_dit* h, const lens_weight* ws, int n_w) {
         }
       if (cudaMemcpy(sw.b_w13, stage.data(), 2 * kMlp * 4, cudaMemcpyHostToDevice) != cudaSuccess)
         return LENS_ERR_CUDA;
-      if ((st = put_bf16(sw.w2, w2, (size_t)D * kMlp))) return st;
+      if ((st = put_block_weight(h, sw.w2, &sw.q_w2, w2, D, kMlp))) return st;
       sw.has_b_w2 = any_nonzero_bf16(L.get(mlp + ".w2.bias", {D}, false), D);
       if ((st = put_f32(sw.b_w2, L.get(mlp + ".w2.bias", {D}, false), D, 0.f, stage))) return st;
     }
@@ -413,8 +466,20 @@ static lens_status make_weight_maps(lens_dit* h) {
   const int D = kHidden;
   bool ok = encode_tmap_bf16(&h->t_txt_in, h->w_txt_in, D, kTxtLayers * kTxtDim, kTxtLayers * kTxtDim, kBnTxtIn) &&
             encode_tmap_bf16(&h->t_img_in, h->w_img_in, D, 2 * kInCh, 2 * kInCh, kBnImgIn) &&
-            encode_tmap_bf16(&h->t_proj, h->w_proj, kInCh, D, D, kBnProj) &&
-            encode_tmap_bf16(&h->t_mod, h->w_mod, h->modw, D, D, 128);
+            encode_tmap_bf16(&h->t_proj, h->w_proj, kInCh, D, D, kBnProj);
+  if (h->w4) {
+    auto qmaps = [](QW& q, uint64_t rows, uint64_t k, uint32_t box) {
+      return encode_tmap_w4_codes(&q.tq, q.codes, rows, k, box) && encode_tmap_w4_scales(&q.ts, q.scales, rows, k, box);
+    };
+    ok = ok && encode_tmap_bf16(&h->t_no, h->w_no, 2 * D, D, D, 128) &&
+         qmaps(h->q_mod, (uint64_t)h->cfg.num_blocks * kModPerBlock, D, 128);
+    for (auto& b : h->blk)
+      for (auto& s : b.s)     // 4-bit block GEMMs run on single CTAs: the B box is the whole tile width
+        ok = ok && qmaps(s.q_qkv, 3 * D, D, kBnQkv) && qmaps(s.q_out, D, D, kBnOut) &&
+             qmaps(s.q_w13, 2 * kMlp, D, kBnW13) && qmaps(s.q_w2, D, kMlp, kBnW2);
+    return ok ? LENS_OK : LENS_ERR_CUDA;
+  }
+  ok = ok && encode_tmap_bf16(&h->t_mod, h->w_mod, h->modw, D, D, 128);
   for (auto& b : h->blk)
     for (auto& s : b.s)
       // block GEMMs run on CTA pairs: each CTA stages half of the B tile
@@ -474,6 +539,21 @@ static lens_status compute_modulation(lens_dit* h, const float* t, int T, cudaSt
   a.p[0].ld_out = h->modw;
   a.p[0].bias = h->b_mod;
   a.p[0].n_valid = T;
+  if (h->w4) {
+    // 4-bit block AdaLN rows, then the bf16 norm_out rows into the same buffer
+    const int mrows = h->cfg.num_blocks * kModPerBlock;
+    a.p[0].M = mrows;
+    LENS_LAUNCH(h, LENS_KERNEL_GEMM_MOD, st, launch_gemm_w4(Tpad, EPI_F32_T, true, nullptr, &tb, &h->q_mod.tq, &h->q_mod.ts, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, a, h->sms, st));
+    GemmArgs a2 = make_args(h->err);
+    a2.num_problems = 1;
+    a2.p[0] = base_problem(2 * kHidden, Tpad, kHidden);
+    a2.p[0].out_f32 = h->mod + mrows;
+    a2.p[0].ld_out = h->modw;
+    a2.p[0].bias = h->b_mod + mrows;
+    a2.p[0].n_valid = T;
+    LENS_LAUNCH(h, LENS_KERNEL_GEMM_MOD, st, launch_gemm(Tpad, EPI_F32_T, &h->t_no, &tb, nullptr, nullptr, nullptr, nullptr, a2, h->sms, st));
+    return LENS_OK;
+  }
   LENS_LAUNCH(h, LENS_KERNEL_GEMM_MOD, st, launch_gemm(Tpad, EPI_F32_T, &h->t_mod, &tb, nullptr, nullptr, nullptr, nullptr, a, h->sms, st));
   return LENS_OK;
 }
@@ -566,8 +646,13 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       p.eps = eps;
       a.p[s] = p;
     }
-    LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_pair(kBnQkv, EPI_QKV, &am.a_img, &wi.t_qkv, np > 1 ? &am.a_txt : nullptr,
-                          np > 1 ? &wt.t_qkv : nullptr, nullptr, nullptr, a, h->sms, st));
+    if (h->w4)
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_w4(kBnQkv, EPI_QKV, false, &am.a_img, nullptr, &wi.q_qkv.tq, &wi.q_qkv.ts,
+                            np > 1 ? &am.a_txt : nullptr, nullptr, np > 1 ? &wt.q_qkv.tq : nullptr, np > 1 ? &wt.q_qkv.ts : nullptr,
+                            nullptr, nullptr, a, h->sms, st));
+    else
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_pair(kBnQkv, EPI_QKV, &am.a_img, &wi.t_qkv, np > 1 ? &am.a_txt : nullptr,
+                            np > 1 ? &wt.t_qkv : nullptr, nullptr, nullptr, a, h->sms, st));
   }
   LENS_LAUNCH(h, LENS_KERNEL_ATTENTION, st, launch_joint_attention(h->q, h->k, h->v, B, kHeads, Nt, Ni, h->o_txt, h->o_img, tl, h->err, st));
   {
@@ -584,8 +669,13 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       p.rows_per_batch = s == 0 ? Ni : Nt;
       a.p[s] = p;
     }
-    LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm_pair(kBnOut, EPI_RESID, &am.o_img, &wi.t_out, np > 1 ? &am.o_txt : nullptr,
-                          np > 1 ? &wt.t_out : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
+    if (h->w4)
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm_w4(kBnOut, EPI_RESID, false, &am.o_img, nullptr, &wi.q_out.tq, &wi.q_out.ts,
+                            np > 1 ? &am.o_txt : nullptr, nullptr, np > 1 ? &wt.q_out.tq : nullptr, np > 1 ? &wt.q_out.ts : nullptr,
+                            &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
+    else
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm_pair(kBnOut, EPI_RESID, &am.o_img, &wi.t_out, np > 1 ? &am.o_txt : nullptr,
+                            np > 1 ? &wt.t_out : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
   }
   // MLP branch
   {
@@ -603,8 +693,13 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       p.bias = w.has_b_w13 ? w.b_w13 : nullptr;
       a.p[s] = p;
     }
-    LENS_LAUNCH(h, LENS_KERNEL_GEMM_W13, st, launch_gemm_pair(kBnW13, EPI_SWIGLU, &am.a_img, &wi.t_w13, np > 1 ? &am.a_txt : nullptr,
-                          np > 1 ? &wt.t_w13 : nullptr, &am.uo_img, np > 1 ? &am.uo_txt : nullptr, a, h->sms, st));
+    if (h->w4)
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_W13, st, launch_gemm_w4(kBnW13, EPI_SWIGLU, false, &am.a_img, nullptr, &wi.q_w13.tq, &wi.q_w13.ts,
+                            np > 1 ? &am.a_txt : nullptr, nullptr, np > 1 ? &wt.q_w13.tq : nullptr, np > 1 ? &wt.q_w13.ts : nullptr,
+                            &am.uo_img, np > 1 ? &am.uo_txt : nullptr, a, h->sms, st));
+    else
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_W13, st, launch_gemm_pair(kBnW13, EPI_SWIGLU, &am.a_img, &wi.t_w13, np > 1 ? &am.a_txt : nullptr,
+                            np > 1 ? &wt.t_w13 : nullptr, &am.uo_img, np > 1 ? &am.uo_txt : nullptr, a, h->sms, st));
   }
   {
     GemmArgs a = make_args(h->err);
@@ -620,8 +715,13 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       p.rows_per_batch = s == 0 ? Ni : Nt;
       a.p[s] = p;
     }
-    LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm_pair(kBnW2, EPI_RESID, &am.u_img, &wi.t_w2, np > 1 ? &am.u_txt : nullptr,
-                          np > 1 ? &wt.t_w2 : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
+    if (h->w4)
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm_w4(kBnW2, EPI_RESID, false, &am.u_img, nullptr, &wi.q_w2.tq, &wi.q_w2.ts,
+                            np > 1 ? &am.u_txt : nullptr, nullptr, np > 1 ? &wt.q_w2.tq : nullptr, np > 1 ? &wt.q_w2.ts : nullptr,
+                            &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
+    else
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm_pair(kBnW2, EPI_RESID, &am.u_img, &wi.t_w2, np > 1 ? &am.u_txt : nullptr,
+                            np > 1 ? &wt.t_w2 : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
   }
   return LENS_OK;
 }
@@ -677,6 +777,7 @@ static lens_status check_model_fields(const lens_dit_config* c) {
       c->freq_dim != d.freq_dim)
     return LENS_ERR_UNSUPPORTED;
   if (c->num_blocks < 1 || c->num_blocks > 48) return LENS_ERR_UNSUPPORTED;
+  if (c->weight_bits != 16 && c->weight_bits != 4) return LENS_ERR_UNSUPPORTED;
   if (!(c->eps > 0.f) || !isfinite(c->eps)) return LENS_ERR_INVALID_ARG;
   if (c->max_batch < 1 || c->max_img_tokens < 1 || c->max_txt_tokens < 0 || c->max_timesteps < 1 ||
       c->max_timesteps > kMaxTimesteps)
@@ -779,6 +880,7 @@ lens_status lens_dit_default_config(lens_dit_config* c) {
   c->max_img_tokens = 4096;
   c->max_txt_tokens = 256;
   c->max_timesteps = 64;
+  c->weight_bits = 16;
   return LENS_OK;
 }
 
@@ -790,6 +892,7 @@ lens_status lens_dit_create(const lens_dit_config* cfg, const lens_weight* w, in
   if (s) return s;
   lens_dit* h = new lens_dit();
   h->cfg = *cfg;
+  h->w4 = cfg->weight_bits == 4;
   h->modw = (int64_t)cfg->num_blocks * kModPerBlock + 2 * kHidden;
   if (cudaGetDevice(&h->device) != cudaSuccess) {
     delete h;
@@ -819,7 +922,18 @@ lens_status lens_dit_create(const lens_dit_config* cfg, const lens_weight* w, in
   sb = Bump();
   sb.base = reinterpret_cast<uintptr_t>(h->ws);
   layout_workspace(h, sb);
+  // weight_bits = 4: one bf16 matrix at a time is staged on the device and quantized
+  if (h->w4 && cudaMalloc(&h->wstage, kStageElems * 2) != cudaSuccess) {
+    cudaGetLastError();
+    lens_dit_destroy(h);
+    return LENS_ERR_OOM;
+  }
   s = load_weights(h, w, n_w);
+  if (h->wstage) {
+    cudaDeviceSynchronize();
+    cudaFree(h->wstage);
+    h->wstage = nullptr;
+  }
   if (s == LENS_OK) s = make_weight_maps(h);
   if (s == LENS_OK && cudaMemsetAsync(h->err, 0, sizeof(int), (cudaStream_t)stream) != cudaSuccess)
     s = LENS_ERR_CUDA;
@@ -837,6 +951,7 @@ void lens_dit_destroy(lens_dit* h) {
   cudaDeviceSynchronize();
   drop_sample_graph(h);
   for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
+  if (h->wstage) cudaFree(h->wstage);
   if (h->ws) cudaFree(h->ws);
   if (h->warena) cudaFree(h->warena);
   delete h;
@@ -1139,6 +1254,37 @@ lens_status lens_op_rmsnorm_modulate(const float* x, int M, int rows_per_batch, 
     return LENS_ERR_INVALID_ARG;
   LENS_CUDA(launch_rmsnorm_modulate(x, M, rows_per_batch, shift, scale, mod_stride, eps,
                                     reinterpret_cast<__nv_bfloat16*>(y), (cudaStream_t)stream));
+  return LENS_OK;
+}
+
+lens_status lens_op_quantize_w4(const uint16_t* w, int64_t rows, int64_t k, uint8_t* codes, uint32_t* scales,
+                                void* stream) {
+  if (!w || !codes || !scales) return LENS_ERR_INVALID_ARG;
+  if (rows < 1 || k < 64 || k % 64) return LENS_ERR_SHAPE;
+  if (reinterpret_cast<uintptr_t>(codes) & 15) return LENS_ERR_INVALID_ARG;
+  LENS_CUDA(launch_quantize_w4(w, rows, k, codes, scales, rows, (cudaStream_t)stream));
+  return LENS_OK;
+}
+
+lens_status lens_op_gemm_w4(const uint16_t* A, const uint8_t* codes, const uint32_t* scales, const float* bias,
+                            float* C, int M, int N, int K, void* stream) {
+  if (!A || !codes || !scales || !C) return LENS_ERR_INVALID_ARG;
+  if (M < 1 || N < 128 || K < 64 || K % 64 || N % 128) return LENS_ERR_SHAPE;
+  const int bn = N % 256 == 0 ? 256 : 128;
+  CUtensorMap ta, tq, ts, tc;
+  if (!encode_tmap_bf16(&ta, A, M, K, K, 128) || !encode_tmap_w4_codes(&tq, codes, N, K, bn) ||
+      !encode_tmap_w4_scales(&ts, scales, N, K, bn) || !encode_tmap_out(&tc, C, 4, M, N, N))
+    return LENS_ERR_INVALID_ARG;
+  int* err = op_err_ptr();
+  if (!err) return LENS_ERR_CUDA;
+  GemmArgs a = make_args(err);
+  a.num_problems = 1;
+  a.p[0] = base_problem(M, N, K);
+  a.p[0].out_f32 = C;
+  a.p[0].ld_out = N;
+  a.p[0].bias = bias;
+  LENS_CUDA(launch_gemm_w4(bn, EPI_F32, false, &ta, nullptr, &tq, &ts, nullptr, nullptr, nullptr, nullptr, &tc,
+                           nullptr, a, device_sms(), (cudaStream_t)stream));
   return LENS_OK;
 }
 

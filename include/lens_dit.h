@@ -78,6 +78,12 @@ typedef struct lens_dit_config {
   int max_img_tokens;    /* grid_h * grid_w */
   int max_txt_tokens;
   int max_timesteps;     /* distinct timesteps whose modulation is kept at once */
+  int weight_bits;       /* 16: bf16 weights.  4: int4 weight-only ("从提示词到成图：
+                            Lens-3.8B-4bit完整管线解析", section 4): every Linear inside the
+                            blocks (qkv, to_out / to_add_out, w1 / w2 / w3, img_mod /
+                            txt_mod) quantized at create (lens_op_quantize_w4's format),
+                            img_in, txt_in, proj_out, the timestep MLP and norm_out kept
+                            in bf16; about 2.35 GB of weights instead of 8.2 GB */
 } lens_dit_config;
 
 /* One named weight tensor, host bf16, row-major [out, in] for Linear weights.
@@ -286,6 +292,25 @@ LENS_API lens_status lens_op_rope_table(int grid_h, int grid_w, int n_txt, float
 LENS_API lens_status lens_op_rmsnorm_modulate(const float* x, int M, int rows_per_batch,
                                      const float* shift, const float* scale, int64_t mod_stride,
                                      float eps, uint16_t* y, void* stream);
+
+/* int4 weight-only ("从提示词到成图：Lens-3.8B-4bit完整管线解析", section 4: 4-bit
+ * weights, group size 64).  lens_op_quantize_w4 quantizes a bf16 weight w [rows, k]
+ * (dev, k a multiple of 64) per group of 64 along k: scale = bf16((max - min) / 15),
+ * bias = bf16(min), code = clamp(rint((w - bias) / scale), 0, 15) in fp32 (0 where
+ * scale = 0); w ~ scale * code + bias.  Caller-owned outputs:
+ *   codes  dev uint8 [rows, k / 2], 16-byte aligned: 32-bit word j of a row holds
+ *          the codes of k in [8j, 8j + 8); the code of k = 8j + 2i sits in bits
+ *          [4i, 4i + 4), that of k = 8j + 2i + 1 in bits [16 + 4i, 20 + 4i)
+ *   scales dev uint32 [k / 64, rows]: group g of row r at [g][r], bf16 scale in the
+ *          low half, bf16 bias in the high half.
+ * lens_op_gemm_w4: C[M,N] = A[M,K] W[N,K]^T (+ bias) with W given as codes/scales
+ * of that layout (rows = N, k = K), widened to bf16 in shared memory before the
+ * tcgen05 MMA; A dev bf16 [M, K], bias dev fp32 [N] or NULL, C dev fp32 [M, N].
+ * N a multiple of 128, K of 64.  Errors: INVALID_ARG (NULL, misaligned), SHAPE. */
+LENS_API lens_status lens_op_quantize_w4(const uint16_t* w, int64_t rows, int64_t k, uint8_t* codes,
+                                         uint32_t* scales, void* stream);
+LENS_API lens_status lens_op_gemm_w4(const uint16_t* A, const uint8_t* codes, const uint32_t* scales,
+                                     const float* bias, float* C, int M, int N, int K, void* stream);
 
 /* Plain bf16 GEMM on the tcgen05 tensor cores: C[M,N] = A[M,K] B[N,K]^T (+ bias),
  * fp32 out.  A, B dev bf16 K-contiguous; bias dev fp32 [N] or NULL; C dev fp32.
