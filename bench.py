@@ -2,7 +2,7 @@
 """Throughput of the Lens MMDiT denoiser + flow-matching Euler sampler on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload turbo_1024] [--impl lens|reference]
-                    [--cfg-rescale PHI] [--shift-mu MU]
+                    [--cfg-rescale PHI] [--shift-mu MU] [--weight-bits 16|4]
 
 One step = one `lens_sample_euler_ex` call on seeded synthetic inputs: noise, text
 input head, timestep/AdaLN modulation for every step, S denoiser forwards of 48
@@ -17,7 +17,8 @@ streamed by every forward, so the working set is far larger than L2 (126 MB).
 Multi-GPU (torchrun): independent replicas, one sample stream per GPU, no data
 exchange (weak scaling).  --impl reference times the CPU oracle instead.
 --cfg-rescale / --shift-mu time the sampler variants (norm-rescaled CFG, shifted
-time grid); without them the call is the plain sampler.
+time grid); without them the call is the plain sampler.  --weight-bits 4 runs the
+int4 weight-only model (block Linears 4-bit, group 64).
 """
 from __future__ import annotations
 
@@ -256,6 +257,8 @@ def main():
                     help="norm-rescaled CFG weight phi in [0, 1] (0: plain CFG)")
     ap.add_argument("--shift-mu", type=float, default=None,
                     help="shifted time grid with this mu (default: uniform grid)")
+    ap.add_argument("--weight-bits", type=int, default=16, choices=[16, 4],
+                    help="4: int4 weight-only block Linears (group 64), quantized at create")
     args = ap.parse_args()
     wl = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -266,6 +269,9 @@ def main():
               "forward_rows": wl.batch * (2 if wl.guidance != 1.0 else 1),
               "l2": "inputs larger than L2: 8.2 GB of weights streamed by every forward",
               "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+    if args.weight_bits != 16:
+        config["weight_bits"] = args.weight_bits
+        config["l2"] = "inputs larger than L2: 2.35 GB of 4-bit block weights streamed by every forward"
     if args.cfg_rescale != 0.0 or args.shift_mu is not None:
         config["sampler_variant"] = {"cfg_rescale": args.cfg_rescale, "shift_mu": args.shift_mu}
 
@@ -295,6 +301,7 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
     cfg = L.lens_dit_default_config()
     rows = config["forward_rows"]
     cfg.max_batch, cfg.max_img_tokens, cfg.max_txt_tokens = rows, wl.n_img, wl.n_txt
+    cfg.weight_bits = args.weight_bits
     h = L.lens_dit_create(cfg, weights)
     del weights
     seed = wl.seed + 1000 * rank

@@ -81,24 +81,32 @@ constexpr int kW4Threads = 320;
 
 // Widen one k block of the 4-bit operand (QROWS rows) into the bf16 tile at dst
 // (128-byte rows, 16-byte chunk c of row n stored at chunk c ^ (n & 7)).  tid in [0, 128).
+// Work item = half a row (32 codes, 16 bytes): one 16-byte code load and one scale
+// load feed four 16-byte stores; a quarter warp stores 8 distinct chunk positions.
 template <int QROWS>
 __device__ __forceinline__ void dequant_block(const uint32_t* __restrict__ qc, const uint32_t* __restrict__ qs,
                                               uint8_t* dst, int tid) {
   const uint32_t k128 = 0x43004300u;                   // bf16 pair (128, 128)
-#pragma unroll 4
-  for (int c = tid; c < QROWS * 8; c += 128) {
-    const int n = c >> 3, wi = c & 7;
-    const uint32_t x = qc[c];
+  static_assert((QROWS * 2) % 128 == 0, "work items must split evenly over the 128 threads");
+#pragma unroll 2
+  for (int it = tid; it < QROWS * 2; it += 128) {
+    const int n = it >> 1, half = it & 1;
+    const uint4 x4 = reinterpret_cast<const uint4*>(qc)[it];
     const uint32_t sbw = qs[n];
     const uint32_t s2 = __byte_perm(sbw, 0, 0x1010), b2 = __byte_perm(sbw, 0, 0x3232);
-    uint32_t o[4];
+    const uint32_t xs[4] = {x4.x, x4.y, x4.z, x4.w};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t v = ((x >> (4 * j)) & 0x000F000Fu) | k128;      // (128 + q_2j, 128 + q_2j+1), exact
-      asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(v) : "r"(v), "r"(k128));
-      asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(o[j]) : "r"(v), "r"(s2), "r"(b2));
+    for (int i = 0; i < 4; ++i) {
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t v = ((xs[i] >> (4 * j)) & 0x000F000Fu) | k128;   // (128 + q_2j, 128 + q_2j+1), exact
+        asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(v) : "r"(v), "r"(k128));
+        asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(o[j]) : "r"(v), "r"(s2), "r"(b2));
+      }
+      const int wi = half * 4 + i;
+      *reinterpret_cast<uint4*>(dst + n * 128 + ((wi ^ (n & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    *reinterpret_cast<uint4*>(dst + n * 128 + ((wi ^ (n & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
