@@ -83,18 +83,28 @@ constexpr int kW4Threads = 320;
 // (128-byte rows, 16-byte chunk c of row n stored at chunk c ^ (n & 7)).  tid in [0, 128).
 // Work item = half a row (32 codes, 16 bytes): one 16-byte code load and one scale
 // load feed four 16-byte stores; a quarter warp stores 8 distinct chunk positions.
+// A thread's items are independent: all their loads are issued before any math.
 template <int QROWS>
 __device__ __forceinline__ void dequant_block(const uint32_t* __restrict__ qc, const uint32_t* __restrict__ qs,
                                               uint8_t* dst, int tid) {
   const uint32_t k128 = 0x43004300u;                   // bf16 pair (128, 128)
+  constexpr int kItems = QROWS * 2 / 128;              // half rows per thread
   static_assert((QROWS * 2) % 128 == 0, "work items must split evenly over the 128 threads");
-#pragma unroll 2
-  for (int it = tid; it < QROWS * 2; it += 128) {
+  // every item's loads first, so their latencies overlap
+  uint4 x4[kItems];
+  uint32_t sbw[kItems];
+#pragma unroll
+  for (int u = 0; u < kItems; ++u) {
+    const int it = tid + 128 * u;
+    x4[u] = reinterpret_cast<const uint4*>(qc)[it];
+    sbw[u] = qs[it >> 1];
+  }
+#pragma unroll
+  for (int u = 0; u < kItems; ++u) {
+    const int it = tid + 128 * u;
     const int n = it >> 1, half = it & 1;
-    const uint4 x4 = reinterpret_cast<const uint4*>(qc)[it];
-    const uint32_t sbw = qs[n];
-    const uint32_t s2 = __byte_perm(sbw, 0, 0x1010), b2 = __byte_perm(sbw, 0, 0x3232);
-    const uint32_t xs[4] = {x4.x, x4.y, x4.z, x4.w};
+    const uint32_t s2 = __byte_perm(sbw[u], 0, 0x1010), b2 = __byte_perm(sbw[u], 0, 0x3232);
+    const uint32_t xs[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       uint32_t o[4];
