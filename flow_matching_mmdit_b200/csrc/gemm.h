@@ -46,8 +46,10 @@ cudaError_t launch_quantize_w4(const void* w_bf16, int64_t rows, int64_t k, uint
 // (the N side, weights [N, K]) is 4-bit, A0/A1 are bf16 maps as for launch_gemm;
 // quant_a = true: A (the M side, weights of the swap-AB modulation GEMM) is 4-bit
 // and B0 is a bf16 map.  Q*/S* are the codes / scales maps (box rows = bn for B,
-// 128 for A).  Same problems, epilogues and output maps as launch_gemm.
-cudaError_t launch_gemm_w4(int bn, int epi, bool quant_a, const CUtensorMap* A0, const CUtensorMap* B0,
+// 128 for A).  bm = 128, or 256 with a 4-bit B (one widened B tile feeds two 128-row
+// MMAs; instantiated for bn = 128).  Same problems, epilogues and output maps as
+// launch_gemm.
+cudaError_t launch_gemm_w4(int bm, int bn, int epi, bool quant_a, const CUtensorMap* A0, const CUtensorMap* B0,
                            const CUtensorMap* Q0, const CUtensorMap* S0, const CUtensorMap* A1, const CUtensorMap* B1,
                            const CUtensorMap* Q1, const CUtensorMap* S1, const CUtensorMap* C0, const CUtensorMap* C1,
                            GemmArgs& args, int sms, cudaStream_t st);

@@ -23,6 +23,9 @@ namespace {
 // the largest block weight staged at create with weight_bits = 4 (one stream's AdaLN)
 constexpr size_t kStageElems = (size_t)kModPerStream * kHidden;
 
+// 4-bit w1|w3: 256 x 128 tiles (one widened B tile feeds two 128-row MMAs)
+constexpr int kBnW13W4 = 128;
+
 constexpr int kBnQkv = 192, kBnOut = 192, kBnW13 = 256, kBnW2 = 192, kBnImgIn = 256, kBnTxtIn = 128,
               kBnProj = 128;
 
@@ -476,7 +479,7 @@ static lens_status make_weight_maps(lens_dit* h) {
     for (auto& b : h->blk)
       for (auto& s : b.s)     // 4-bit block GEMMs run on single CTAs: the B box is the whole tile width
         ok = ok && qmaps(s.q_qkv, 3 * D, D, kBnQkv) && qmaps(s.q_out, D, D, kBnOut) &&
-             qmaps(s.q_w13, 2 * kMlp, D, kBnW13) && qmaps(s.q_w2, D, kMlp, kBnW2);
+             qmaps(s.q_w13, 2 * kMlp, D, kBnW13W4) && qmaps(s.q_w2, D, kMlp, kBnW2);
     return ok ? LENS_OK : LENS_ERR_CUDA;
   }
   ok = ok && encode_tmap_bf16(&h->t_mod, h->w_mod, h->modw, D, D, 128);
@@ -543,7 +546,7 @@ static lens_status compute_modulation(lens_dit* h, const float* t, int T, cudaSt
     // 4-bit block AdaLN rows, then the bf16 norm_out rows into the same buffer
     const int mrows = h->cfg.num_blocks * kModPerBlock;
     a.p[0].M = mrows;
-    LENS_LAUNCH(h, LENS_KERNEL_GEMM_MOD, st, launch_gemm_w4(Tpad, EPI_F32_T, true, nullptr, &tb, &h->q_mod.tq, &h->q_mod.ts, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, a, h->sms, st));
+    LENS_LAUNCH(h, LENS_KERNEL_GEMM_MOD, st, launch_gemm_w4(128, Tpad, EPI_F32_T, true, nullptr, &tb, &h->q_mod.tq, &h->q_mod.ts, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, a, h->sms, st));
     GemmArgs a2 = make_args(h->err);
     a2.num_problems = 1;
     a2.p[0] = base_problem(2 * kHidden, Tpad, kHidden);
@@ -647,7 +650,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     if (h->w4)
-      LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_w4(kBnQkv, EPI_QKV, false, &am.a_img, nullptr, &wi.q_qkv.tq, &wi.q_qkv.ts,
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_w4(128, kBnQkv, EPI_QKV, false, &am.a_img, nullptr, &wi.q_qkv.tq, &wi.q_qkv.ts,
                             np > 1 ? &am.a_txt : nullptr, nullptr, np > 1 ? &wt.q_qkv.tq : nullptr, np > 1 ? &wt.q_qkv.ts : nullptr,
                             nullptr, nullptr, a, h->sms, st));
     else
@@ -670,7 +673,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     if (h->w4)
-      LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm_w4(kBnOut, EPI_RESID, false, &am.o_img, nullptr, &wi.q_out.tq, &wi.q_out.ts,
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm_w4(128, kBnOut, EPI_RESID, false, &am.o_img, nullptr, &wi.q_out.tq, &wi.q_out.ts,
                             np > 1 ? &am.o_txt : nullptr, nullptr, np > 1 ? &wt.q_out.tq : nullptr, np > 1 ? &wt.q_out.ts : nullptr,
                             &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
     else
@@ -694,7 +697,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     if (h->w4)
-      LENS_LAUNCH(h, LENS_KERNEL_GEMM_W13, st, launch_gemm_w4(kBnW13, EPI_SWIGLU, false, &am.a_img, nullptr, &wi.q_w13.tq, &wi.q_w13.ts,
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_W13, st, launch_gemm_w4(256, kBnW13W4, EPI_SWIGLU, false, &am.a_img, nullptr, &wi.q_w13.tq, &wi.q_w13.ts,
                             np > 1 ? &am.a_txt : nullptr, nullptr, np > 1 ? &wt.q_w13.tq : nullptr, np > 1 ? &wt.q_w13.ts : nullptr,
                             &am.uo_img, np > 1 ? &am.uo_txt : nullptr, a, h->sms, st));
     else
@@ -716,7 +719,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     if (h->w4)
-      LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm_w4(kBnW2, EPI_RESID, false, &am.u_img, nullptr, &wi.q_w2.tq, &wi.q_w2.ts,
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm_w4(128, kBnW2, EPI_RESID, false, &am.u_img, nullptr, &wi.q_w2.tq, &wi.q_w2.ts,
                             np > 1 ? &am.u_txt : nullptr, nullptr, np > 1 ? &wt.q_w2.tq : nullptr, np > 1 ? &wt.q_w2.ts : nullptr,
                             &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
     else
@@ -1271,6 +1274,7 @@ lens_status lens_op_gemm_w4(const uint16_t* A, const uint8_t* codes, const uint3
   if (!A || !codes || !scales || !C) return LENS_ERR_INVALID_ARG;
   if (M < 1 || N < 128 || K < 64 || K % 64 || N % 128) return LENS_ERR_SHAPE;
   const int bn = N % 256 == 0 ? 256 : 128;
+  const int bm = bn == 128 && M >= 256 ? 256 : 128;   // 256-row tiles with the 128-wide B tile
   CUtensorMap ta, tq, ts, tc;
   if (!encode_tmap_bf16(&ta, A, M, K, K, 128) || !encode_tmap_w4_codes(&tq, codes, N, K, bn) ||
       !encode_tmap_w4_scales(&ts, scales, N, K, bn) || !encode_tmap_out(&tc, C, 4, M, N, N))
@@ -1283,7 +1287,7 @@ lens_status lens_op_gemm_w4(const uint16_t* A, const uint8_t* codes, const uint3
   a.p[0].out_f32 = C;
   a.p[0].ld_out = N;
   a.p[0].bias = bias;
-  LENS_CUDA(launch_gemm_w4(bn, EPI_F32, false, &ta, nullptr, &tq, &ts, nullptr, nullptr, nullptr, nullptr, &tc,
+  LENS_CUDA(launch_gemm_w4(bm, bn, EPI_F32, false, &ta, nullptr, &tq, &ts, nullptr, nullptr, nullptr, nullptr, &tc,
                            nullptr, a, device_sms(), (cudaStream_t)stream));
   return LENS_OK;
 }

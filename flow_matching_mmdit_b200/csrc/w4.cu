@@ -56,11 +56,13 @@ __global__ void quantize_w4_kernel(const __nv_bfloat16* __restrict__ w, int64_t 
 }
 
 // ------------------------------------------------------------------ GEMM configuration
-template <int BN, int EPI, bool QA>
+// MH = 128-row halves of the M tile (2: one widened B tile feeds two M = 128 MMAs,
+// halving the widening per MMA flop; B side only).
+template <int BN, int EPI, bool QA, int MH = 1>
 struct GemmW4Cfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr int QROWS = QA ? BM : BN;                       // rows of the 4-bit operand tile
-  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t A_BYTES = MH * BM * BK * 2;
   static constexpr uint32_t B_BYTES = BN * BK * 2;
   static constexpr uint32_t QC_BYTES = QROWS * 32;                 // codes of one k block
   static constexpr uint32_t QS_BYTES = ((QROWS * 4 + 127) / 128) * 128;
@@ -72,9 +74,11 @@ struct GemmW4Cfg {
   static constexpr uint32_t BAR_BYTES = 512;
   static constexpr uint32_t BUDGET = 232448 - 1024 - BAR_BYTES - EPI_BYTES - AUX_BYTES;
   static constexpr int STAGES = (BUDGET / STAGE_BYTES) > 8 ? 8 : (BUDGET / STAGE_BYTES);
-  static constexpr uint32_t TMEM_COLS = pow2_at_least(2 * BN);
+  static constexpr uint32_t TMEM_COLS = pow2_at_least(2 * MH * BN);
   static constexpr size_t SMEM = 1024 + size_t(STAGES) * STAGE_BYTES + EPI_BYTES + AUX_BYTES + BAR_BYTES;
   static_assert(STAGES >= 2, "shared memory too small for two stages");
+  static_assert(MH == 1 || (MH == 2 && !QA), "two M halves only with a 4-bit B");
+  static_assert(2 * MH * BN <= 512, "two accumulators must fit TMEM");
 };
 
 constexpr int kW4Threads = 320;
@@ -120,6 +124,14 @@ __device__ __forceinline__ void dequant_block(const uint32_t* __restrict__ qc, c
   }
 }
 
+template <int MH>
+__device__ __forceinline__ void w4_decode(const GemmArgs& a, int t, int bn, int& pi, int& m0, int& n0) {
+  if (MH == 2)
+    decode_tile2(a, t, bn, pi, m0, n0);       // 256-row tiles
+  else
+    decode_tile(a, t, bn, pi, m0, n0);
+}
+
 // ------------------------------------------------------------------ kernel
 // Warp roles (320 threads):
 //   warp 0      TMA: the bf16 operand tile (A when QA is false, else B), the codes and
@@ -129,15 +141,16 @@ __device__ __forceinline__ void dequant_block(const uint32_t* __restrict__ qc, c
 //   warps 6..9  widen the 4-bit operand of each stage into its bf16 slot, make the
 //               stores visible to the tensor core (async proxy), arrive on bfull
 // bfull is arrived only after full completed, so it also covers the TMA bytes.
-template <int BN, int EPI, bool QA>
+template <int BN, int EPI, bool QA, int MH>
 __global__ void __launch_bounds__(kW4Threads, 1)
     gemm_w4_kernel(const __grid_constant__ CUtensorMap tmX0, const __grid_constant__ CUtensorMap tmQ0,
                    const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmX1,
                    const __grid_constant__ CUtensorMap tmQ1, const __grid_constant__ CUtensorMap tmS1,
                    const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1,
                    const __grid_constant__ GemmArgs args) {
-  using C = GemmW4Cfg<BN, EPI, QA>;
+  using C = GemmW4Cfg<BN, EPI, QA, MH>;
   constexpr int STAGES = C::STAGES;
+  constexpr uint32_t A_HALF = C::A_BYTES / MH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -200,7 +213,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < args.total_tiles && ok; t += gridDim.x) {
         int pi, m0, n0;
-        decode_tile(args, t, BN, pi, m0, n0);
+        w4_decode<MH>(args, t, BN, pi, m0, n0);
         const CUtensorMap* mX = pi ? &tmX1 : &tmX0;
         const CUtensorMap* mQ = pi ? &tmQ1 : &tmQ0;
         const CUtensorMap* mS = pi ? &tmS1 : &tmS0;
@@ -212,10 +225,13 @@ __global__ void __launch_bounds__(kW4Threads, 1)
             break;
           }
           mbar_expect_tx(&full[stage], C::TX_BYTES);
-          if (QA)
+          if (QA) {
             tma_load_2d(sB + stage * C::B_BYTES, mX, &full[stage], kb * C::BK, n0);
-          else
-            tma_load_2d(sA + stage * C::A_BYTES, mX, &full[stage], kb * C::BK, m0);
+          } else {
+#pragma unroll
+            for (int h = 0; h < MH; ++h)
+              tma_load_2d(sA + stage * C::A_BYTES + h * A_HALF, mX, &full[stage], kb * C::BK, m0 + 128 * h);
+          }
           tma_load_2d(sQc + stage * C::QC_BYTES, mQ, &full[stage], kb * 32, q0);
           tma_load_2d(sQs + stage * C::QS_BYTES, mS, &full[stage], q0, kb);
           issued[stage] = true;
@@ -240,24 +256,27 @@ __global__ void __launch_bounds__(kW4Threads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < args.total_tiles && ok; t += gridDim.x, ++li) {
         int pi, m0, n0;
-        decode_tile(args, t, BN, pi, m0, n0);
+        w4_decode<MH>(args, t, BN, pi, m0, n0);
         const int kblocks = args.p[pi].K / C::BK;
         const uint32_t acc = li & 1;
         const uint32_t use = li >> 1;
         if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t d_tmem = tmem_base + acc * MH * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&bfull[stage], phase, args.err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t ad = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES));
           const uint64_t bd = umma_desc_sw128(smem_u32(sB + stage * C::B_BYTES));
 #pragma unroll
-          for (int k = 0; k < C::BK / 16; ++k)
-            umma_bf16(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int h = 0; h < MH; ++h) {
+            const uint64_t ad = umma_desc_sw128(smem_u32(sA + stage * C::A_BYTES + h * A_HALF));
+#pragma unroll
+            for (int k = 0; k < C::BK / 16; ++k)
+              umma_bf16(d_tmem + h * BN, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           umma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -276,15 +295,18 @@ __global__ void __launch_bounds__(kW4Threads, 1)
     int li = 0;
     for (int t = blockIdx.x; t < args.total_tiles; t += gridDim.x, ++li) {
       int pi, m0, n0;
-      decode_tile(args, t, BN, pi, m0, n0);
+      w4_decode<MH>(args, t, BN, pi, m0, n0);
       const uint32_t acc = li & 1;
       const uint32_t use = li >> 1;
       if (!mbar_wait(&tfull[acc], use & 1, args.err)) break;
       tc_fence_after();
-      const int row0 = m0 + quarter * 32;
-      const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
-      epilogue_tile<BN, EPI>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots, slot,
-                             sAux + pi * 128);
+#pragma unroll 1
+      for (int h = 0; h < MH; ++h) {
+        const int row0 = m0 + 128 * h + quarter * 32;
+        const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * MH * BN + h * BN;
+        epilogue_tile<BN, EPI>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots, slot,
+                               sAux + pi * 128);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -299,7 +321,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < args.total_tiles && ok; t += gridDim.x) {
       int pi, m0, n0;
-      decode_tile(args, t, BN, pi, m0, n0);
+      w4_decode<MH>(args, t, BN, pi, m0, n0);
       const int kblocks = args.p[pi].K / C::BK;
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait(&full[stage], phase, args.err)) {
@@ -328,20 +350,20 @@ __global__ void __launch_bounds__(kW4Threads, 1)
   }
 }
 
-template <int BN, int EPI, bool QA>
+template <int BN, int EPI, bool QA, int MH>
 cudaError_t launch_w4_one(const CUtensorMap& X0, const CUtensorMap& Q0, const CUtensorMap& S0, const CUtensorMap& X1,
                           const CUtensorMap& Q1, const CUtensorMap& S1, const CUtensorMap& C0, const CUtensorMap& C1,
                           const GemmArgs& args, int sms, cudaStream_t st) {
-  using C = GemmW4Cfg<BN, EPI, QA>;
+  using C = GemmW4Cfg<BN, EPI, QA, MH>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_w4_kernel<BN, EPI, QA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(gemm_w4_kernel<BN, EPI, QA, MH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int grid = args.total_tiles < sms ? args.total_tiles : sms;
-  gemm_w4_kernel<BN, EPI, QA><<<grid, kW4Threads, C::SMEM, st>>>(X0, Q0, S0, X1, Q1, S1, C0, C1, args);
+  gemm_w4_kernel<BN, EPI, QA, MH><<<grid, kW4Threads, C::SMEM, st>>>(X0, Q0, S0, X1, Q1, S1, C0, C1, args);
   return cudaGetLastError();
 }
 
@@ -359,11 +381,12 @@ cudaError_t launch_quantize_w4(const void* w_bf16, int64_t rows, int64_t k, uint
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_w4(int bn, int epi, bool quant_a, const CUtensorMap* A0, const CUtensorMap* B0,
+cudaError_t launch_gemm_w4(int bm, int bn, int epi, bool quant_a, const CUtensorMap* A0, const CUtensorMap* B0,
                            const CUtensorMap* Q0, const CUtensorMap* S0, const CUtensorMap* A1, const CUtensorMap* B1,
                            const CUtensorMap* Q1, const CUtensorMap* S1, const CUtensorMap* C0, const CUtensorMap* C1,
                            GemmArgs& args, int sms, cudaStream_t st) {
-  finalize_problems(args, bn, 128);
+  if (bm != 128 && (bm != 256 || quant_a)) return cudaErrorInvalidValue;
+  finalize_problems(args, bn, bm);
   if (args.total_tiles == 0) return cudaSuccess;
   const CUtensorMap* X0 = quant_a ? B0 : A0;
   const CUtensorMap* X1 = quant_a ? B1 : A1;
@@ -375,17 +398,19 @@ cudaError_t launch_gemm_w4(int bn, int epi, bool quant_a, const CUtensorMap* A0,
   const CUtensorMap& s1 = S1 ? *S1 : *S0;
   const CUtensorMap& c0 = C0 ? *C0 : *X0;
   const CUtensorMap& c1 = C1 ? *C1 : c0;
-#define LENS_W4_CASE(BN_, EPI_, QA_)                                                                        \
-  if (bn == BN_ && epi == EPI_ && quant_a == QA_)                                                           \
-    return launch_w4_one<BN_, EPI_, QA_>(*X0, *Q0, *S0, x1, q1, s1, c0, c1, args, sms, st);
-  LENS_W4_CASE(256, EPI_F32, false)
-  LENS_W4_CASE(128, EPI_F32, false)
-  LENS_W4_CASE(192, EPI_QKV, false)
-  LENS_W4_CASE(192, EPI_RESID, false)
-  LENS_W4_CASE(256, EPI_SWIGLU, false)
-  LENS_W4_CASE(16, EPI_F32_T, true)
-  LENS_W4_CASE(32, EPI_F32_T, true)
-  LENS_W4_CASE(64, EPI_F32_T, true)
+#define LENS_W4_CASE(BM_, BN_, EPI_, QA_)                                                                   \
+  if (bm == BM_ && bn == BN_ && epi == EPI_ && quant_a == QA_)                                              \
+    return launch_w4_one<BN_, EPI_, QA_, BM_ / 128>(*X0, *Q0, *S0, x1, q1, s1, c0, c1, args, sms, st);
+  LENS_W4_CASE(128, 256, EPI_F32, false)
+  LENS_W4_CASE(128, 128, EPI_F32, false)
+  LENS_W4_CASE(256, 128, EPI_F32, false)
+  LENS_W4_CASE(128, 192, EPI_QKV, false)
+  LENS_W4_CASE(128, 192, EPI_RESID, false)
+  LENS_W4_CASE(128, 256, EPI_SWIGLU, false)
+  LENS_W4_CASE(256, 128, EPI_SWIGLU, false)
+  LENS_W4_CASE(128, 16, EPI_F32_T, true)
+  LENS_W4_CASE(128, 32, EPI_F32_T, true)
+  LENS_W4_CASE(128, 64, EPI_F32_T, true)
 #undef LENS_W4_CASE
   return cudaErrorInvalidValue;
 }
