@@ -24,7 +24,7 @@ namespace {
 constexpr size_t kStageElems = (size_t)kModPerStream * kHidden;
 
 // 4-bit w1|w3: 256 x 128 tiles (one widened B tile feeds two 128-row MMAs)
-constexpr int kBnW13W4 = 128;
+constexpr int kBnW13W4 = 128, kBnQkvW4 = 128;
 
 constexpr int kBnQkv = 192, kBnOut = 192, kBnW13 = 256, kBnW2 = 192, kBnImgIn = 256, kBnTxtIn = 128,
               kBnProj = 128;
@@ -478,7 +478,7 @@ static lens_status make_weight_maps(lens_dit* h) {
          qmaps(h->q_mod, (uint64_t)h->cfg.num_blocks * kModPerBlock, D, 128);
     for (auto& b : h->blk)
       for (auto& s : b.s)     // 4-bit block GEMMs run on single CTAs: the B box is the whole tile width
-        ok = ok && qmaps(s.q_qkv, 3 * D, D, kBnQkv) && qmaps(s.q_out, D, D, kBnOut) &&
+        ok = ok && qmaps(s.q_qkv, 3 * D, D, kBnQkvW4) && qmaps(s.q_out, D, D, kBnOut) &&
              qmaps(s.q_w13, 2 * kMlp, D, kBnW13W4) && qmaps(s.q_w2, D, kMlp, kBnW2);
     return ok ? LENS_OK : LENS_ERR_CUDA;
   }
@@ -650,7 +650,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     if (h->w4)
-      LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_w4(128, kBnQkv, EPI_QKV, false, &am.a_img, nullptr, &wi.q_qkv.tq, &wi.q_qkv.ts,
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_w4(256, kBnQkvW4, EPI_QKV, false, &am.a_img, nullptr, &wi.q_qkv.tq, &wi.q_qkv.ts,
                             np > 1 ? &am.a_txt : nullptr, nullptr, np > 1 ? &wt.q_qkv.tq : nullptr, np > 1 ? &wt.q_qkv.ts : nullptr,
                             nullptr, nullptr, a, h->sms, st));
     else

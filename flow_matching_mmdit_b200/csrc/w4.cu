@@ -405,6 +405,7 @@ cudaError_t launch_gemm_w4(int bm, int bn, int epi, bool quant_a, const CUtensor
   LENS_W4_CASE(128, 128, EPI_F32, false)
   LENS_W4_CASE(256, 128, EPI_F32, false)
   LENS_W4_CASE(128, 192, EPI_QKV, false)
+  LENS_W4_CASE(256, 128, EPI_QKV, false)
   LENS_W4_CASE(128, 192, EPI_RESID, false)
   LENS_W4_CASE(128, 256, EPI_SWIGLU, false)
   LENS_W4_CASE(256, 128, EPI_SWIGLU, false)
