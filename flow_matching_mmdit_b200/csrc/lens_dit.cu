@@ -23,8 +23,9 @@ namespace {
 // the largest block weight staged at create with weight_bits = 4 (one stream's AdaLN)
 constexpr size_t kStageElems = (size_t)kModPerStream * kHidden;
 
-// 4-bit w1|w3: 256 x 128 tiles (one widened B tile feeds two 128-row MMAs)
-constexpr int kBnW13W4 = 128, kBnQkvW4 = 128;
+// 4-bit block GEMMs on 256-row tiles (one widened B tile feeds two 128-row MMAs):
+// 128 wide for w1|w3 and QKV, 96 wide for the 1536-wide to_out and w2 (272 tiles)
+constexpr int kBnW13W4 = 128, kBnQkvW4 = 128, kBnResW4 = 96;
 
 constexpr int kBnQkv = 192, kBnOut = 192, kBnW13 = 256, kBnW2 = 192, kBnImgIn = 256, kBnTxtIn = 128,
               kBnProj = 128;
@@ -478,8 +479,8 @@ static lens_status make_weight_maps(lens_dit* h) {
          qmaps(h->q_mod, (uint64_t)h->cfg.num_blocks * kModPerBlock, D, 128);
     for (auto& b : h->blk)
       for (auto& s : b.s)     // 4-bit block GEMMs run on single CTAs: the B box is the whole tile width
-        ok = ok && qmaps(s.q_qkv, 3 * D, D, kBnQkvW4) && qmaps(s.q_out, D, D, kBnOut) &&
-             qmaps(s.q_w13, 2 * kMlp, D, kBnW13W4) && qmaps(s.q_w2, D, kMlp, kBnW2);
+        ok = ok && qmaps(s.q_qkv, 3 * D, D, kBnQkvW4) && qmaps(s.q_out, D, D, kBnResW4) &&
+             qmaps(s.q_w13, 2 * kMlp, D, kBnW13W4) && qmaps(s.q_w2, D, kMlp, kBnResW4);
     return ok ? LENS_OK : LENS_ERR_CUDA;
   }
   ok = ok && encode_tmap_bf16(&h->t_mod, h->w_mod, h->modw, D, D, 128);
@@ -673,7 +674,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     if (h->w4)
-      LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm_w4(128, kBnOut, EPI_RESID, false, &am.o_img, nullptr, &wi.q_out.tq, &wi.q_out.ts,
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm_w4(256, kBnResW4, EPI_RESID, false, &am.o_img, nullptr, &wi.q_out.tq, &wi.q_out.ts,
                             np > 1 ? &am.o_txt : nullptr, nullptr, np > 1 ? &wt.q_out.tq : nullptr, np > 1 ? &wt.q_out.ts : nullptr,
                             &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
     else
@@ -719,7 +720,7 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       a.p[s] = p;
     }
     if (h->w4)
-      LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm_w4(128, kBnW2, EPI_RESID, false, &am.u_img, nullptr, &wi.q_w2.tq, &wi.q_w2.ts,
+      LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm_w4(256, kBnResW4, EPI_RESID, false, &am.u_img, nullptr, &wi.q_w2.tq, &wi.q_w2.ts,
                             np > 1 ? &am.u_txt : nullptr, nullptr, np > 1 ? &wt.q_w2.tq : nullptr, np > 1 ? &wt.q_w2.ts : nullptr,
                             &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
     else

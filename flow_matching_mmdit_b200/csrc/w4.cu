@@ -92,20 +92,22 @@ template <int QROWS>
 __device__ __forceinline__ void dequant_block(const uint32_t* __restrict__ qc, const uint32_t* __restrict__ qs,
                                               uint8_t* dst, int tid) {
   const uint32_t k128 = 0x43004300u;                   // bf16 pair (128, 128)
-  constexpr int kItems = QROWS * 2 / 128;              // half rows per thread
-  static_assert((QROWS * 2) % 128 == 0, "work items must split evenly over the 128 threads");
+  constexpr int kItems = (QROWS * 2 + 127) / 128;      // half rows per thread (the last may be partial)
   // every item's loads first, so their latencies overlap
   uint4 x4[kItems];
   uint32_t sbw[kItems];
 #pragma unroll
   for (int u = 0; u < kItems; ++u) {
     const int it = tid + 128 * u;
-    x4[u] = reinterpret_cast<const uint4*>(qc)[it];
-    sbw[u] = qs[it >> 1];
+    if (it < QROWS * 2) {
+      x4[u] = reinterpret_cast<const uint4*>(qc)[it];
+      sbw[u] = qs[it >> 1];
+    }
   }
 #pragma unroll
   for (int u = 0; u < kItems; ++u) {
     const int it = tid + 128 * u;
+    if (it >= QROWS * 2) break;
     const int n = it >> 1, half = it & 1;
     const uint32_t s2 = __byte_perm(sbw[u], 0, 0x1010), b2 = __byte_perm(sbw[u], 0, 0x3232);
     const uint32_t xs[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
@@ -407,6 +409,7 @@ cudaError_t launch_gemm_w4(int bm, int bn, int epi, bool quant_a, const CUtensor
   LENS_W4_CASE(128, 192, EPI_QKV, false)
   LENS_W4_CASE(256, 128, EPI_QKV, false)
   LENS_W4_CASE(128, 192, EPI_RESID, false)
+  LENS_W4_CASE(256, 96, EPI_RESID, false)
   LENS_W4_CASE(128, 256, EPI_SWIGLU, false)
   LENS_W4_CASE(256, 128, EPI_SWIGLU, false)
   LENS_W4_CASE(128, 16, EPI_F32_T, true)
