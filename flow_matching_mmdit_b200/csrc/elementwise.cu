@@ -123,7 +123,8 @@ __global__ void rope_table_kernel(int gh, int gw, int n_txt, int ntok, float2* _
 // One warp per row of 1536 fp32: y = (1 + scale) * x * rsqrt(mean(x^2) + eps) + shift.
 // Up to two independent segments (the image and the text stream of a block) share
 // one launch: rows [0, s0.M) belong to segment 0, the next s1.M rows to segment 1.
-__global__ void rmsnorm_modulate_kernel(RmsSeg s0, RmsSeg s1, float eps) {
+// 64 registers (4 blocks of 256 per SM): the 4352 rows of a 1024^2 block fit one wave.
+__global__ void __launch_bounds__(256, 4) rmsnorm_modulate_kernel(RmsSeg s0, RmsSeg s1, float eps) {
   int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const RmsSeg* sg = &s0;
