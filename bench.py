@@ -2,7 +2,7 @@
 """Throughput of the Lens MMDiT denoiser + flow-matching Euler sampler on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload turbo_1024] [--impl lens|reference]
-                    [--cfg-rescale PHI] [--shift-mu MU] [--weight-bits 16|4]
+                    [--cfg-rescale PHI] [--shift-mu MU] [--weight-bits 16|4] [--txt-valid T]
 
 One step = one `lens_sample_euler_ex` call on seeded synthetic inputs: noise, text
 input head, timestep/AdaLN modulation for every step, S denoiser forwards of 48
@@ -18,7 +18,8 @@ Multi-GPU (torchrun): independent replicas, one sample stream per GPU, no data
 exchange (weak scaling).  --impl reference times the CPU oracle instead.
 --cfg-rescale / --shift-mu time the sampler variants (norm-rescaled CFG, shifted
 time grid); without them the call is the plain sampler.  --weight-bits 4 runs the
-int4 weight-only model (block Linears 4-bit, group 64).
+int4 weight-only model (block Linears 4-bit, group 64).  --txt-valid T marks all but the
+first T text tokens of every sample as padding (masked keys in attention).
 """
 from __future__ import annotations
 
@@ -257,6 +258,8 @@ def main():
                     help="norm-rescaled CFG weight phi in [0, 1] (0: plain CFG)")
     ap.add_argument("--shift-mu", type=float, default=None,
                     help="shifted time grid with this mu (default: uniform grid)")
+    ap.add_argument("--txt-valid", type=int, default=None,
+                    help="valid text tokens per sample (the rest are padding, masked in attention)")
     ap.add_argument("--weight-bits", type=int, default=16, choices=[16, 4],
                     help="4: int4 weight-only block Linears (group 64), quantized at create")
     args = ap.parse_args()
@@ -269,6 +272,8 @@ def main():
               "forward_rows": wl.batch * (2 if wl.guidance != 1.0 else 1),
               "l2": "inputs larger than L2: 8.2 GB of weights streamed by every forward",
               "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+    if args.txt_valid is not None:
+        config["txt_valid"] = args.txt_valid
     if args.weight_bits != 16:
         config["weight_bits"] = args.weight_bits
         config["l2"] = "inputs larger than L2: 2.35 GB of 4-bit block weights streamed by every forward"
@@ -315,8 +320,10 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
     if args.shift_mu is not None:
         opt.time_shift, opt.shift_mu = 1, args.shift_mu
 
+    lens = None if args.txt_valid is None else [args.txt_valid] * wl.batch
+
     def sample(text):
-        L.lens_sample_euler_ex(h, text, None, None, None, wl.batch, wl.n_txt, wl.height_px, wl.width_px, wl.steps,
+        L.lens_sample_euler_ex(h, text, lens, None, lens, wl.batch, wl.n_txt, wl.height_px, wl.width_px, wl.steps,
                                opt, seed, out)
 
     def step():

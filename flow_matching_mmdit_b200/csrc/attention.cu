@@ -9,6 +9,7 @@
 // rows past N are computed on zero-filled queries and never stored.
 #include "gemm.h"
 #include "kernels.cuh"
+#include "smem_attr.h"
 
 namespace lens {
 
@@ -365,12 +366,10 @@ cudaError_t launch_joint_attention(const __nv_bfloat16* q, const __nv_bfloat16* 
       !encode_tmap_bf16_3d(&tk, k, 64, N, (uint64_t)B * heads, 128) ||
       !encode_tmap_bf16_3d(&tv, v, 64, N, (uint64_t)B * heads, 128))
     return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(tc::joint_attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)tc::SMEM);
+  static std::atomic<uint64_t> attr{0};
+  {
+    const cudaError_t e = ensure_smem_limit(tc::joint_attention_tc_kernel, (int)tc::SMEM, attr);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   dim3 grid((N + tc::TILES * tc::BQ - 1) / (tc::TILES * tc::BQ), heads, B);
   const float scale_log2 = 0.125f * 1.4426950408889634f;

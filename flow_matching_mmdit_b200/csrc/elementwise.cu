@@ -5,6 +5,7 @@
 #include <math.h>
 
 #include "kernels.cuh"
+#include "smem_attr.h"
 
 namespace lens {
 
@@ -360,11 +361,10 @@ cudaError_t launch_small_linear(const float* x, int T, int K, const __nv_bfloat1
                                 bool silu_in, float* out, __nv_bfloat16* silu_out_bf16, int silu_rows,
                                 cudaStream_t st) {
   const size_t smem = (size_t)8 * K * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(small_linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
+  static std::atomic<uint64_t> attr{0};
+  {
+    const cudaError_t e = ensure_smem_limit(small_linear_kernel, 65536, attr);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   small_linear_kernel<<<(N + 7) / 8, 256, smem, st>>>(x, T, K, W, bias, N, silu_in ? 1 : 0, out, silu_out_bf16,
                                                        silu_rows);

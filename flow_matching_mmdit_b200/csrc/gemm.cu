@@ -3,6 +3,7 @@
 
 #include "gemm.h"
 #include "gemm_tc.cuh"
+#include "smem_attr.h"
 
 namespace lens {
 
@@ -29,12 +30,10 @@ template <int BN, int EPI>
 cudaError_t launch_one(const CUtensorMap& A0, const CUtensorMap& B0, const CUtensorMap& A1, const CUtensorMap& B1,
                        const CUtensorMap& C0, const CUtensorMap& C1, const GemmArgs& args, int sms, cudaStream_t st) {
   using C = GemmCfg<BN, EPI>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::SMEM);
+  static std::atomic<uint64_t> attr{0};
+  {
+    const cudaError_t e = ensure_smem_limit(gemm_tc_kernel<BN, EPI>, (int)C::SMEM, attr);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const int grid = args.total_tiles < sms ? args.total_tiles : sms;
   gemm_tc_kernel<BN, EPI><<<grid, 192, C::SMEM, st>>>(A0, B0, A1, B1, C0, C1, args);
@@ -46,12 +45,10 @@ cudaError_t launch_pair(const CUtensorMap& A0, const CUtensorMap& B0, const CUte
                         const CUtensorMap& C0, const CUtensorMap& C1, const GemmArgs& args, int sms,
                         cudaStream_t st) {
   using C = Gemm2Cfg<BN, EPI>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm2_tc_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::SMEM);
+  static std::atomic<uint64_t> attr{0};
+  {
+    const cudaError_t e = ensure_smem_limit(gemm2_tc_kernel<BN, EPI>, (int)C::SMEM, attr);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const int pairs = args.total_tiles < sms / 2 ? args.total_tiles : sms / 2;
   gemm2_tc_kernel<BN, EPI><<<2 * pairs, 192, C::SMEM, st>>>(A0, B0, A1, B1, C0, C1, args);

@@ -10,6 +10,7 @@
 // the bf16 GEMM's (gemm_tc.cuh).
 #include "gemm.h"
 #include "gemm_tc.cuh"
+#include "smem_attr.h"
 
 namespace lens {
 
@@ -357,12 +358,10 @@ cudaError_t launch_w4_one(const CUtensorMap& X0, const CUtensorMap& Q0, const CU
                           const CUtensorMap& Q1, const CUtensorMap& S1, const CUtensorMap& C0, const CUtensorMap& C1,
                           const GemmArgs& args, int sms, cudaStream_t st) {
   using C = GemmW4Cfg<BN, EPI, QA, MH>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_w4_kernel<BN, EPI, QA, MH>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  static std::atomic<uint64_t> attr{0};
+  {
+    const cudaError_t e = ensure_smem_limit(gemm_w4_kernel<BN, EPI, QA, MH>, (int)C::SMEM, attr);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const int grid = args.total_tiles < sms ? args.total_tiles : sms;
   gemm_w4_kernel<BN, EPI, QA, MH><<<grid, kW4Threads, C::SMEM, st>>>(X0, Q0, S0, X1, Q1, S1, C0, C1, args);
