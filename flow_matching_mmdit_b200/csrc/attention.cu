@@ -49,19 +49,28 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
+
 // ============================================================ tcgen05 version
 // One CTA per (256 query rows = two 128-row tiles X = 0, 1; head; batch row).
-// Warp roles (320 threads):
-//   warps 0..3  softmax of tile 0, warps 4..7 softmax of tile 1: one query row per
-//               thread; S_X is read from TMEM into registers and released at once,
-//               so the tensor cores compute S_X for the next keys while this tile's
-//               exponentials run, and the two tiles ping-pong on the tensor cores
-//   warp 8      TMA: both Q tiles once, then K and V tiles of 128 keys (3 stages)
-//   warp 9      UMMA issuer: S_X = Q_X K_j^T (M=128, N=128, K=64) and
-//               O_X += P_X V_j (M=128, N=64, K=128) with P_X read from TMEM.
-//               A wait in this thread stalls until its queued UMMAs are accepted,
-//               so the waits S_0 and S_1 need (K/V stage, both S slots released)
-//               are taken back to back: the queue drains once for them.
+// Warp roles (608 threads):
+//   warps 0..15 softmax, eight warps per tile (X = warp / 8): warp (quarter q, half
+//               h) owns TMEM lanes 32q + 16h + [0, 16) and reads S_X with the
+//               16-lane shape, so each thread holds two query rows (r and r + 8) and
+//               32 of the 128 keys of each, and the four threads of a row combine
+//               their maxima with two shuffles.  Four softmax warps per SMSP and 64
+//               scores per thread (not 128) leave room to hide the exponential and
+//               TMEM latencies.  S_X is released as soon as it is in registers, so
+//               the tensor cores compute S_X for the next keys meanwhile.
+//   warp 16     TMA: both Q tiles once, then K and V tiles of 128 keys (3 stages)
+//   warp 17     S issuer: S_X = Q_X K_j^T (M=128, N=128, K=64), each tile as soon
+//               as its S slot is released
+//   warp 18     P V issuer: O_X += P_X V_j (M=128, N=64, K=128) with P_X in TMEM.
+//               A wait in an issuing thread stalls until that thread's queued UMMAs
+//               are accepted, so the two kinds of MMA come from two threads: a P V
+//               wait does not hold back the next S, nor the reverse.
+// Tile 1 starts its first exponentials only when tile 0 has finished its own: the
+// two tiles then keep alternating on the exponential unit instead of contending
+// for it in phase.
 // The running max m and sum l of each row live in registers; O_X is rescaled in
 // TMEM only when m grows by more than 2^8 (softmax is invariant to the subtracted
 // constant, so a stale max is exact up to rounding).
@@ -72,7 +81,7 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 namespace tc {
 
 constexpr int BQ = 128, BKV = 128, STAGES = 3, TILES = 2;
-constexpr int THREADS = 320;
+constexpr int THREADS = 608;
 constexpr uint32_t Q_BYTES = BQ * 64 * 2;          // 16 KB per query tile
 constexpr uint32_t KV_BYTES = BKV * 64 * 2;        // 16 KB each for K and V
 constexpr uint32_t OFF_Q = 0;
@@ -89,6 +98,7 @@ struct Bars {
   uint64_t s_free[TILES];    // softmax -> MMA: S_X read into registers
   uint64_t p_full[TILES];    // softmax -> MMA: P_X written, O_X rescaled
   uint64_t pv_done[TILES];   // MMA -> softmax: O_X += P_X V finished
+  uint64_t stagger;          // tile 0 -> tile 1: tile 0 finished its first exponentials
   uint32_t tmem_slot;
 };
 
@@ -116,20 +126,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&bar.q_full, 1);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bar.kv_full[s], 1);
-      mbar_init(&bar.kv_empty[s], 1);
+      mbar_init(&bar.kv_empty[s], 2);
     }
     for (int x = 0; x < TILES; ++x) {
       mbar_init(&bar.s_full[x], 1);
-      mbar_init(&bar.s_free[x], 4);
-      mbar_init(&bar.p_full[x], 4);
+      mbar_init(&bar.s_free[x], 8);
+      mbar_init(&bar.p_full[x], 8);
       mbar_init(&bar.pv_done[x], 1);
     }
+    mbar_init(&bar.stagger, 8);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
-  if (warp == 9) {
+  if (warp == 17) {
     tmem_alloc(&bar.tmem_slot, 512);
     tmem_relinquish();
   }
@@ -138,7 +149,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bar.tmem_slot;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       uint32_t last_parity[STAGES] = {0, 0, 0};
@@ -165,183 +176,215 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (issued[s]) mbar_wait_drain(&bar.kv_full[s], last_parity[s]);
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ---------------------------------------------------------------- UMMA issuer
+  } else if (warp == 17) {
+    // ---------------------------------------------------------------- S issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16(128, BKV);
-      constexpr uint32_t idesc_pv = umma_idesc_bf16_bmn(128, 64);
       bool ok = mbar_wait(&bar.q_full, 0, err);
       tc_fence_after();
-      for (int j = 0; ok && j <= nkv; ++j) {
-        if (j < nkv) {
-          const int s = j % STAGES;
-          // every wait S_0[j] and S_1[j] need, back to back: only the first drains the queue
-          ok = mbar_wait(&bar.kv_full[s], (j / STAGES) & 1, err) &&
-               (j == 0 || (mbar_wait(&bar.s_free[0], (j - 1) & 1, err) && mbar_wait(&bar.s_free[1], (j - 1) & 1, err)));
-          if (!ok) break;
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int s = j % STAGES;
+        ok = mbar_wait(&bar.kv_full[s], (j / STAGES) & 1, err);
+        if (!ok) break;
+        const uint64_t kdesc = umma_desc_sw128(smem_u32(sKV + s * 2 * KV_BYTES));
+#pragma unroll
+        for (int x = 0; x < TILES; ++x) {
+          if (j > 0 && !mbar_wait(&bar.s_free[x], (j - 1) & 1, err)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint64_t kdesc = umma_desc_sw128(smem_u32(sKV + s * 2 * KV_BYTES));
+          const uint64_t qdesc = umma_desc_sw128(smem_u32(sQ + x * Q_BYTES));
 #pragma unroll
-          for (int x = 0; x < TILES; ++x) {
-            const uint64_t qdesc = umma_desc_sw128(smem_u32(sQ + x * Q_BYTES));
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              umma_bf16(tmem + x * 128, qdesc + 2 * k, kdesc + 2 * k, idesc_s, k > 0 ? 1u : 0u);
-            umma_commit(&bar.s_full[x]);
-          }
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(tmem + x * 128, qdesc + 2 * k, kdesc + 2 * k, idesc_s, k > 0 ? 1u : 0u);
+          umma_commit(&bar.s_full[x]);
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int s = jj % STAGES;
-          const uint32_t vbase = smem_u32(sKV + s * 2 * KV_BYTES + KV_BYTES);
+        if (!ok) break;
+        umma_commit(&bar.kv_empty[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 18) {
+    // ---------------------------------------------------------------- P V issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = umma_idesc_bf16_bmn(128, 64);
+      bool ok = true;
+      for (int jj = 0; ok && jj < nkv; ++jj) {
+        const int s = jj % STAGES;
+        const uint32_t vbase = smem_u32(sKV + s * 2 * KV_BYTES + KV_BYTES);
 #pragma unroll
-          for (int x = 0; x < TILES; ++x) {
-            if (!mbar_wait(&bar.p_full[x], jj & 1, err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {              // 16 keys = 8 TMEM columns of P per step
-              const uint64_t vdesc = umma_desc_sw128_mn(vbase + k * 2048);
-              umma_bf16_ts(tmem + 256 + x * 64, tmem + 384 + x * 64 + 8 * k, vdesc, idesc_pv,
-                           (jj > 0 || k > 0) ? 1u : 0u);
-            }
-            umma_commit(&bar.pv_done[x]);
+        for (int x = 0; x < TILES; ++x) {
+          if (!mbar_wait(&bar.p_full[x], jj & 1, err)) {
+            ok = false;
+            break;
           }
-          if (!ok) break;
-          umma_commit(&bar.kv_empty[s]);
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint64_t vdesc = umma_desc_sw128_mn(vbase + k * 2048);
+            umma_bf16_ts(tmem + 256 + x * 64, tmem + 384 + x * 64 + 8 * k, vdesc, idesc_pv,
+                         (jj > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&bar.pv_done[x]);
         }
+        if (!ok) break;
+        umma_commit(&bar.kv_empty[s]);
       }
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax
-    const int x = warp >> 2;                // query tile
-    const int quarter = warp & 3;           // TMEM lane quarter
-    const int r = quarter * 32 + lane;      // row inside the tile
-    const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
+    // Eight warps per tile: warp (quarter, half) reads TMEM lanes quarter*32 + half*16
+    // + [0, 16); each thread holds rows rlo and rlo + 8, 32 of the 128 keys of each
+    // (columns 8g + cq + {0, 1}); the four threads of a row combine maxima by shuffles.
+    const int x = warp >> 3;
+    const int half = (warp >> 2) & 1;
+    const int quarter = warp & 3;
+    const int rlo = quarter * 32 + half * 16 + (lane >> 2);
+    const uint32_t lane_addr = tmem + (uint32_t(quarter * 32 + half * 16) << 16);
     const uint32_t s_col = x * 128, o_col = 256 + x * 64, p_col = 384 + x * 64;
-    float m = -INFINITY, l = 0.f;
+    const int cq = 2 * (lane & 3);
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      if (!mbar_wait(&bar.s_full[x], j & 1, err)) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.s_full[x], j & 1, err))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float sc[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(lane_addr + s_col + c * 32, *reinterpret_cast<float(*)[32]>(&sc[32 * c]));
+      float sc[64];
+      tmem_ld_16x256b_x16(lane_addr + s_col, sc);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar.s_free[x]);     // S_X may be overwritten now
+      if (lane == 0) mbar_arrive(&bar.s_free[x]);
       if ((j + 1) * BKV > N) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (j * BKV + i >= N) sc[i] = -INFINITY;
-      }
-      if (j * BKV < txt_pad_end && (j + 1) * BKV > txt_valid) {   // padded text keys of this sample
+        for (int g = 0; g < 16; ++g)
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (j * BKV + i >= txt_valid && j * BKV + i < txt_pad_end) sc[i] = -INFINITY;
+          for (int e = 0; e < 2; ++e)
+            if (j * BKV + 8 * g + cq + e >= N) sc[4 * g + e] = sc[4 * g + 2 + e] = -INFINITY;
       }
-      // 8 independent partial maxima (three-input max) keep the dependency chains short
-      float pm[8];
+      if (j * BKV < txt_pad_end && (j + 1) * BKV > txt_valid) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        pm[q] = max3f(sc[q], sc[q + 8], sc[q + 16]);
+        for (int g = 0; g < 16; ++g)
 #pragma unroll
-        for (int t = 3; t < 15; t += 2) pm[q] = max3f(pm[q], sc[q + 8 * t], sc[q + 8 * t + 8]);
-        pm[q] = fmaxf(pm[q], sc[q + 120]);
+          for (int e = 0; e < 2; ++e) {
+            const int key = j * BKV + 8 * g + cq + e;
+            if (key >= txt_valid && key < txt_pad_end) sc[4 * g + e] = sc[4 * g + 2 + e] = -INFINITY;
+          }
       }
-      float mx = max3f(max3f(pm[0], pm[1], pm[2]), max3f(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-      mx *= scale_log2;
-      float corr = 1.f;
-      if (mx > m + kRescaleThreshold) {
-        corr = ex2(m - mx);
-        m = mx;
-      }
-      // every key seen so far masked: m is still -inf and so is every score here
-      const float m_base = m == -INFINITY ? 0.f : m;
-      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-      // x = s log2(e) / 8 - m for two keys per instruction
-      const uint64_t sl2 = f2_pack(scale_log2, scale_log2), mb2 = f2_pack(-m_base, -m_base);
-      uint32_t pk[64];
+      float p0[4], p1[4];
 #pragma unroll
-      for (int i = 0; i < 128; i += 2) {
-        float x0, x1;
-        f2_unpack(f2_fma(f2_pack(sc[i], sc[i + 1]), sl2, mb2), x0, x1);
-        const float e0 = ex2(x0), e1 = ex2(x1);
-        acc2[(i >> 1) & 3] = f2_add(acc2[(i >> 1) & 3], f2_pack(e0, e1));
-        pk[i >> 1] = pack_bf16x2(e0, e1);
+      for (int q = 0; q < 4; ++q) {
+        p0[q] = fmaxf(sc[4 * q], sc[4 * q + 1]);
+        p1[q] = fmaxf(sc[4 * q + 2], sc[4 * q + 3]);
       }
-      float ps[8];
-      f2_unpack(acc2[0], ps[0], ps[1]);
-      f2_unpack(acc2[1], ps[2], ps[3]);
-      f2_unpack(acc2[2], ps[4], ps[5]);
-      f2_unpack(acc2[3], ps[6], ps[7]);
-      const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      l = l * corr + rs;
+#pragma unroll
+      for (int g = 4; g < 16; ++g) {
+        p0[g & 3] = max3f(p0[g & 3], sc[4 * g], sc[4 * g + 1]);
+        p1[g & 3] = max3f(p1[g & 3], sc[4 * g + 2], sc[4 * g + 3]);
+      }
+      float mx0 = max3f(p0[0], p0[1], fmaxf(p0[2], p0[3]));
+      float mx1 = max3f(p1[0], p1[1], fmaxf(p1[2], p1[3]));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2)) * scale_log2;
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2)) * scale_log2;
+      float c0 = 1.f, c1 = 1.f;
+      if (mx0 > m0 + kRescaleThreshold) {
+        c0 = ex2(m0 - mx0);
+        m0 = mx0;
+      }
+      if (mx1 > m1 + kRescaleThreshold) {
+        c1 = ex2(m1 - mx1);
+        m1 = mx1;
+      }
+      const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
+      const uint64_t nb0 = f2_pack(m0 == -INFINITY ? 0.f : -m0, m0 == -INFINITY ? 0.f : -m0);
+      const uint64_t nb1 = f2_pack(m1 == -INFINITY ? 0.f : -m1, m1 == -INFINITY ? 0.f : -m1);
+      if (x == 1 && j == 0 && !__all_sync(0xffffffffu, mbar_wait(&bar.stagger, 0, err))) {
+        ok = false;
+        break;
+      }
+      uint64_t a0[2] = {0ull, 0ull}, a1[2] = {0ull, 0ull};
+      uint32_t pk[32];
+#pragma unroll
+      for (int g = 0; g < 16; ++g) {
+        float x0, x1, x2, x3;
+        f2_unpack(f2_fma(f2_pack(sc[4 * g], sc[4 * g + 1]), sl2, nb0), x0, x1);
+        f2_unpack(f2_fma(f2_pack(sc[4 * g + 2], sc[4 * g + 3]), sl2, nb1), x2, x3);
+        const float e0 = ex2(x0), e1 = ex2(x1), e2 = ex2(x2), e3 = ex2(x3);
+        a0[g & 1] = f2_add(a0[g & 1], f2_pack(e0, e1));
+        a1[g & 1] = f2_add(a1[g & 1], f2_pack(e2, e3));
+        pk[2 * g] = pack_bf16x2(e0, e1);
+        pk[2 * g + 1] = pack_bf16x2(e2, e3);
+      }
+      if (x == 0 && j == 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.stagger);
+      }
+      float s0, s1, s2, s3;
+      f2_unpack(f2_add(a0[0], a0[1]), s0, s1);
+      f2_unpack(f2_add(a1[0], a1[1]), s2, s3);
+      l0 = l0 * c0 + (s0 + s1);
+      l1 = l1 * c1 + (s2 + s3);
       if (j > 0) {
-        if (!mbar_wait(&bar.pv_done[x], (j - 1) & 1, err)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar.pv_done[x], (j - 1) & 1, err))) {
           ok = false;
           break;
         }
         tc_fence_after();
       }
-      // P row r -> TMEM, column c = keys (2c, 2c + 1)
-      tmem_st32_u(lane_addr + p_col, pk);
-      tmem_st32_u(lane_addr + p_col + 32, pk + 32);
-      if (j > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+      tmem_st_16x128b_x16(lane_addr + p_col, pk);
+      if (j > 0 && __any_sync(0xffffffffu, c0 != 1.f || c1 != 1.f)) {
+        float o[32];
+        tmem_ld_16x256b_x8(lane_addr + o_col, o);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float o[32];
-          tmem_ld32(lane_addr + o_col + c * 32, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= corr;
-          tmem_st32(lane_addr + o_col + c * 32, o);
+        for (int g = 0; g < 8; ++g) {
+          o[4 * g] *= c0;
+          o[4 * g + 1] *= c0;
+          o[4 * g + 2] *= c1;
+          o[4 * g + 3] *= c1;
         }
+        tmem_st_16x256b_x8(lane_addr + o_col, o);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.p_full[x]);
     }
-    if (ok && mbar_wait(&bar.pv_done[x], (nkv - 1) & 1, err)) {
+    // row sums: the four threads of a row hold disjoint keys
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    if (__all_sync(0xffffffffu, ok && mbar_wait(&bar.pv_done[x], (nkv - 1) & 1, err))) {
       tc_fence_after();
-      float o0[32], o1[32];
-      tmem_ld32(lane_addr + o_col, o0);
-      tmem_ld32(lane_addr + o_col + 32, o1);
+      float o[32];
+      tmem_ld_16x256b_x8(lane_addr + o_col, o);
       tmem_ld_wait();
-      const int tok = q0 + x * BQ + r;
-      if (tok < N) {
-        const float inv = 1.f / l;
-        const int hid = heads * 64;
-        __nv_bfloat16* dst = tok < n_txt ? out_txt + ((int64_t)b * n_txt + tok) * hid
-                                         : out_img + ((int64_t)b * (N - n_txt) + (tok - n_txt)) * hid;
-        uint4* d4 = reinterpret_cast<uint4*>(dst + h * 64);
+      const int hid = heads * 64;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          d4[q] = make_uint4(pack_bf16x2(o0[8 * q] * inv, o0[8 * q + 1] * inv),
-                             pack_bf16x2(o0[8 * q + 2] * inv, o0[8 * q + 3] * inv),
-                             pack_bf16x2(o0[8 * q + 4] * inv, o0[8 * q + 5] * inv),
-                             pack_bf16x2(o0[8 * q + 6] * inv, o0[8 * q + 7] * inv));
+      for (int rr = 0; rr < 2; ++rr) {
+        const int tok = q0 + x * BQ + rlo + 8 * rr;
+        if (tok < N) {
+          const float inv = 1.f / (rr ? l1 : l0);
+          __nv_bfloat16* dst = tok < n_txt ? out_txt + ((int64_t)b * n_txt + tok) * hid
+                                           : out_img + ((int64_t)b * (N - n_txt) + (tok - n_txt)) * hid;
+          uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + h * 64 + cq);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          d4[4 + q] = make_uint4(pack_bf16x2(o1[8 * q] * inv, o1[8 * q + 1] * inv),
-                                 pack_bf16x2(o1[8 * q + 2] * inv, o1[8 * q + 3] * inv),
-                                 pack_bf16x2(o1[8 * q + 4] * inv, o1[8 * q + 5] * inv),
-                                 pack_bf16x2(o1[8 * q + 6] * inv, o1[8 * q + 7] * inv));
+          for (int g = 0; g < 8; ++g)
+            d32[4 * g] = pack_bf16x2(o[4 * g + 2 * rr] * inv, o[4 * g + 2 * rr + 1] * inv);
+        }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
