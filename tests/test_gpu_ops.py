@@ -132,6 +132,31 @@ def test_joint_attention(B, nt, ni):
     assert np.max(np.abs(got - ref)) < 0.05
 
 
+@pytest.mark.parametrize("nt,ni", [(256, 4096), (7, 333)])
+def test_joint_attention_rows_do_not_depend_on_the_batch(nt, ni):
+    """Each batch row's output bits are the same computed alone or next to another row:
+    no CTA's arithmetic depends on the rest of the launch (the CFG split across ranks
+    is bit-exact against the batched CFG sampler because of it)."""
+    import torch
+    rng = np.random.default_rng(ni + 1)
+    N = nt + ni
+    q, k, v = (f32_to_bf16_bits(rng.standard_normal((2, 24, N, 64)).astype(np.float32) * s) for s in (1.5, 1.5, 1))
+
+    def run(rows):
+        B = len(rows)
+        ot = torch.full((B, nt, 1536), -1, dtype=torch.int16, device="cuda")
+        oi = torch.full((B, ni, 1536), -1, dtype=torch.int16, device="cuda")
+        qs, ks, vs = (dev(np.ascontiguousarray(a[rows])) for a in (q, k, v))
+        L.lens_op_attention(qs, ks, vs, B, nt, ni, ot, oi)
+        _sync()
+        return host(ot), host(oi)
+
+    bt, bi = run([0, 1])
+    for r in (0, 1):
+        at, ai = run([r])
+        assert np.array_equal(at[0], bt[r]) and np.array_equal(ai[0], bi[r])
+
+
 def test_euler_cfg_op():
     import torch
     rng = np.random.default_rng(9)
