@@ -402,15 +402,17 @@ def euler(x: np.ndarray, v: np.ndarray, dt: float) -> np.ndarray:
 
 
 def sample_euler(velocity: Callable[[np.ndarray, float, bool], np.ndarray], x1: np.ndarray,
-                 steps: int, guidance: float, mu: Optional[float] = None, phi: float = 0.0) -> np.ndarray:
+                 steps: int, guidance: float, mu: Optional[float] = None, phi: float = 0.0,
+                 stop_after: Optional[int] = None) -> np.ndarray:
     """Integrate from t = 1 to 0 with S Euler steps.  velocity(x, t, cond) gives the
     conditional (cond=True) or unconditional prediction.  guidance == 1 evaluates the
     conditional model only ([mlx] "guidance 1.0": no doubled forward).  mu shifts the
     time grid (time_grid), phi rescales the guided velocity (cfg_rescaled); with
-    neither, the steps are the uniform 1/S."""
+    neither, the steps are the uniform 1/S.  stop_after = k returns the state after
+    the first k steps of the S-step grid (None = all S)."""
     x = x1
     tg = time_grid(steps, mu)
-    for k in range(steps):
+    for k in range(steps if stop_after is None else min(stop_after, steps)):
         t = float(tg[k])
         dt = 1.0 / steps if mu is None else float(tg[k] - tg[k + 1])
         vc = velocity(x, t, True)
@@ -427,36 +429,36 @@ def sample(W: Weights, dims, E_cond: np.ndarray, E_uncond: Optional[np.ndarray],
            grid_h: int, grid_w: int, steps: int, guidance: float, seed: int,
            blocks: Optional[int] = None, len_cond: Optional[Sequence[int]] = None,
            len_uncond: Optional[Sequence[int]] = None, mu: Optional[float] = None,
-           phi: float = 0.0) -> np.ndarray:
+           phi: float = 0.0, stop_after: Optional[int] = None,
+           trace: Optional[list] = None) -> np.ndarray:
     """Full sampler: seeded noise latent [B, 32, 2h, 2w] -> latent at t = 0.
-    Cond and uncond run as one batch of 2B (cond first) when guidance != 1.
+    The step loop is `sample_euler`; its velocity field is the denoiser `forward` on
+    the patchified latent, with the conditional text for cond and the unconditional
+    text otherwise (rows are independent, so running the two halves as one batch of
+    2B, as the GPU does, computes the same thing).
     READING: unconditional text = zeros of the same shape when E_uncond is None.
     len_cond / len_uncond: valid text lengths per sample (None = all valid).
-    mu: shifted time grid (time_grid); phi: norm-rescaled CFG (cfg_rescaled)."""
+    mu: shifted time grid (time_grid); phi: norm-rescaled CFG (cfg_rescaled);
+    stop_after: return the latent after that many steps of the S-step grid.
+    trace: a list that receives (t, cond, tokens, velocity) for every forward."""
     C, p = dims.latent_channels, dims.patch
     z = noise(seed, B * C * p * grid_h * p * grid_w).reshape(B, C, p * grid_h, p * grid_w)
-    x = z.astype(W.dtype)
     if guidance != 1.0 and E_uncond is None:
         E_uncond = np.zeros_like(E_cond)
     Nt = E_cond.shape[1]
     lc = None if len_cond is None and len_uncond is None else \
         list(len_cond if len_cond is not None else [Nt] * B)
     lu = None if lc is None else list(len_uncond if len_uncond is not None else [Nt] * B)
-    tg = time_grid(steps, mu)
-    for k in range(steps):
-        t = float(tg[k])
-        dt = 1.0 / steps if mu is None else float(tg[k] - tg[k + 1])
+
+    def velocity(x: np.ndarray, t: float, cond: bool) -> np.ndarray:
         X = patchify(x, p)
-        if guidance == 1.0:
-            v = forward(W, dims, X, grid_h, grid_w, E_cond, [t] * B, blocks, txt_len=lc)
-        else:
-            vv = forward(W, dims, np.concatenate([X, X]), grid_h, grid_w,
-                         np.concatenate([E_cond, E_uncond]), [t] * (2 * B), blocks,
-                         txt_len=None if lc is None else lc + lu)
-            v = cfg_combine(vv[:B], vv[B:], guidance) if phi == 0.0 else \
-                cfg_rescaled(vv[:B], vv[B:], guidance, phi)
-        x = euler(x, unpatchify(v, grid_h, grid_w, C, p), dt)
-    return x
+        v = forward(W, dims, X, grid_h, grid_w, E_cond if cond else E_uncond, [t] * B, blocks,
+                    txt_len=lc if cond else lu)
+        if trace is not None:
+            trace.append((t, cond, X, v))
+        return unpatchify(v, grid_h, grid_w, C, p)
+
+    return sample_euler(velocity, z.astype(W.dtype), steps, guidance, mu, phi, stop_after)
 
 
 # ============================================================ int4 weight-only (4-bit page)

@@ -527,3 +527,159 @@ def test_block_padding_has_no_influence(tinyW):
     # the unpadded sample equals the unmasked block
     hu, tu = o.block(tinyW, 0, h_img, h_txt, temb, ang, TINY.heads, TINY.eps)
     assert np.allclose(hi[1], hu[1], atol=1e-12) and not np.allclose(hi[0], hu[0], atol=1e-6)
+
+
+# ------------------------------------------------------------------ closed-form pins of the remaining pieces
+def _silu(x):
+    return x / (1.0 + math.exp(-x))          # the sigmoid-weighted linear unit, by its definition
+
+
+def test_gated_mlp_unit_vector_closed_form():
+    """[blog] "Overview" (gate / up / down of 1536x4096) with the READING w1 = gated branch:
+    unit rows in w1 and w3 pick x_i and x_j, a unit column of w2 routes their product to
+    one output, so that output is silu(x_i) * x_j exactly.  A sum in place of the product,
+    SiLU on the product, or SiLU on the w3 branch all give other numbers here."""
+    D, F = 5, 3
+    w1, w3, w2 = np.zeros((F, D)), np.zeros((F, D)), np.zeros((D, F))
+    w1[0, 1], w3[0, 2], w2[4, 0] = 1.0, 1.0, 1.0        # out_4 = silu(x_1) * x_2
+    w1[1, 2], w3[1, 1], w2[0, 1] = 1.0, 1.0, 1.0        # out_0 = silu(x_2) * x_1 (branches swapped)
+    w1[2, 3], w3[2, 3], w2[2, 2] = 1.0, 1.0, 2.0        # out_2 = 2 silu(x_3) * x_3
+    W = o.Weights({"m.w1.weight": w1, "m.w3.weight": w3, "m.w2.weight": w2,
+                   "m.w2.bias": np.array([0.0, 0.0, 0.0, 0.5, 0.0])})
+    x = np.array([[0.3, 1.0, -2.0, 0.5, 7.0]])
+    y = o.gated_mlp(W, "m", x)[0]
+    expect = [_silu(-2.0) * 1.0, 0.0, 2.0 * _silu(0.5) * 0.5, 0.5, _silu(1.0) * -2.0]
+    assert np.allclose(y, expect, rtol=0, atol=1e-15)
+    assert abs(expect[4] - (-1.4621171572600098)) < 1e-15  # silu(1) = 0.7310585786300049
+
+
+def test_final_layer_closed_form():
+    """[mlx] "Patchify 补丁化与输出投影": norm_out.linear then proj_out.  With zero
+    norm_out weights its bias alone sets (scale, shift) (READING: scale first), and
+    identity rows in proj_out expose (1 + scale) * x / rms(x) + shift column by column.
+    The row [3, -4, 0, 0] has rms 2.5 (eps = 0), so x / rms(x) = [1.2, -1.6, 0, 0]."""
+    D, C = 4, 3
+    proj = np.zeros((C, D))
+    proj[0, 0] = proj[1, 1] = proj[2, 2] = 1.0
+    bias = np.array([1.0, 0.5, -1.0, 2.0, 0.25, -0.5, 3.0, 1.0])   # scale | shift
+    W = o.Weights({"norm_out.linear.weight": np.zeros((2 * D, D)), "norm_out.linear.bias": bias,
+                   "proj_out.weight": proj, "proj_out.bias": np.array([0.0, 0.0, 10.0])})
+    h = np.array([[[3.0, -4.0, 0.0, 0.0], [0.0, 0.0, 5.0, 0.0]]])
+    temb = np.array([[0.7, -1.0, 2.0, 0.0]])
+    v = o.final_layer(W, h, temb, 0.0)[0]
+    # row 0: [(1+1) 1.2 + 0.25, (1+0.5)(-1.6) - 0.5, 0 + 3 + 10]; row 1 has x/rms = [0, 0, 2, 0]
+    assert np.allclose(v[0], [2.65, -2.9, 13.0], rtol=0, atol=1e-14)
+    assert np.allclose(v[1], [0.25, -0.5, 0.0 * 2.0 + 3.0 + 10.0], rtol=0, atol=1e-14)
+    # scale = shift = 0 is the plain RMSNorm
+    W0 = o.Weights({"norm_out.linear.weight": np.zeros((2 * D, D)), "proj_out.weight": proj})
+    assert np.allclose(o.final_layer(W0, h, temb, 0.0)[0, 0], [1.2, -1.6, 0.0], rtol=0, atol=1e-15)
+    # the projection sees SiLU(temb): one unit weight makes scale_0 = 1 + silu(2)
+    wn = np.zeros((2 * D, D))
+    wn[0, 2] = 1.0
+    W1 = o.Weights({"norm_out.linear.weight": wn, "norm_out.linear.bias": bias, "proj_out.weight": proj})
+    assert abs(o.final_layer(W1, h, temb, 0.0)[0, 0, 0] - ((2.0 + _silu(2.0)) * 1.2 + 0.25)) < 1e-14
+
+
+def test_timestep_embedding_mlp_closed_form():
+    """temb = linear_2(SiLU(linear_1(e))) ([mlx] time_text_embed.timestep_embedder).  At
+    t = 0 the features are [1 ... 1, 0 ... 0] (cos 0, sin 0), so unit rows in linear_1
+    (with biases) give known pre-activations and linear_2 routes their SiLUs."""
+    fd, D = 16, 4
+    l1, b1 = np.zeros((D, fd)), np.array([0.0, -3.0, -0.5, 0.0])
+    l1[0, 0] = 1.0                 # cos part: 1          -> silu(1)
+    l1[1, 8] = 1.0                 # sin part: 0, bias -3 -> silu(-3)
+    l1[2, 0] = l1[2, 1] = 1.0      # 2 - 0.5             -> silu(1.5)
+    l2, b2 = np.zeros((D, D)), np.array([0.0, 0.0, 0.0, 1.0])
+    l2[0, 2] = l2[1, 0] = l2[2, 1] = 1.0
+    l2[3, 0] = 2.0
+    p = "time_text_embed.timestep_embedder"
+    W = o.Weights({p + ".linear_1.weight": l1, p + ".linear_1.bias": b1,
+                   p + ".linear_2.weight": l2, p + ".linear_2.bias": b2})
+    temb = o.timestep_embedding(W, np.array([0.0]), fd)[0]
+    s1, sm3, s15 = 0.7310585786300049, -3.0 / (1.0 + math.exp(3.0)), 1.5 / (1.0 + math.exp(-1.5))
+    assert np.allclose(temb, [s15, s1, sm3, 2.0 * s1 + 1.0], rtol=0, atol=1e-15)
+
+
+def _zero_model_with_output_bias(d, b):
+    w = {}
+    for name, shape, _ in weight_specs(d):
+        w[name] = np.zeros(shape)
+    w["proj_out.bias"] = np.asarray(b, np.float64)
+    return o.Weights(w)
+
+
+@pytest.mark.parametrize("steps,mu,guidance", [(1, None, 1.0), (4, None, 1.0), (7, None, 5.0),
+                                               (4, 0.7, 1.0), (7, -0.4, 3.0)])
+def test_sample_constant_field_lands_exactly(steps, mu, guidance):
+    """A model whose only nonzero weight is the proj_out bias b has v = b for every token,
+    t and text, so the sampler returns noise(seed) - unpatchify(b) for any step count and
+    any grid ([paper] "Flow Matching 训练目标": the grid runs from t = 1 to t = 0, so the
+    steps add up to 1).  The expected latent is written out from the patch layout
+    (channel c, patch row r, patch column s at feature 4c + 2r + s)."""
+    d = TINY
+    rng = np.random.default_rng(5)
+    b = rng.standard_normal(d.in_channels)
+    W = _zero_model_with_output_bias(d, b)
+    gh, gw, B, seed = 2, 3, 2, 123
+    E = rng.standard_normal((B, 3, d.txt_layers, d.txt_dim))
+    x = o.sample(W, d, E, None, B, gh, gw, steps, guidance, seed, mu=mu)
+    C = d.latent_channels
+    z = o.noise(seed, B * C * 2 * gh * 2 * gw).astype(np.float64).reshape(B, C, 2 * gh, 2 * gw)
+    shift = np.empty((C, 2 * gh, 2 * gw))
+    for c in range(C):
+        for yy in range(2 * gh):
+            for xx in range(2 * gw):
+                shift[c, yy, xx] = b[4 * c + 2 * (yy % 2) + (xx % 2)]
+    assert np.allclose(x, z - shift[None], rtol=0, atol=1e-12)
+
+
+def test_sample_wiring_with_guidance(tinyW):
+    """Two CFG steps on the tiny random model, written out from the pinned parts:
+    x1 = z - (1/2) g(z, 1), x2 = x1 - (1/2) g(x1, 1/2) with g = u + s (c - u), where c and
+    u are the forward on the patchified latent with the conditional and unconditional
+    text.  A swapped cond/uncond, a wrong t or a wrong dt all fail here."""
+    d = TINY
+    rng = np.random.default_rng(9)
+    gh, gw, B, seed, s = 2, 2, 1, 77, 3.0
+    Ec = rng.standard_normal((B, 3, d.txt_layers, d.txt_dim))
+    Eu = rng.standard_normal((B, 3, d.txt_layers, d.txt_dim))
+    C = d.latent_channels
+
+    def f(x, t, E):
+        return o.unpatchify(o.forward(tinyW, d, o.patchify(x), gh, gw, E, [t] * B), gh, gw, C)
+
+    def g(x, t):
+        c, u = f(x, t, Ec), f(x, t, Eu)
+        assert np.linalg.norm(c - u) > 1e-3 * np.linalg.norm(c)   # text reaches the image
+        return u + s * (c - u)
+
+    z = o.noise(seed, B * C * 4 * gh * gw).astype(np.float64).reshape(B, C, 2 * gh, 2 * gw)
+    x1 = z - 0.5 * g(z, 1.0)
+    x2 = x1 - 0.5 * g(x1, 0.5)
+    trace = []
+    got = o.sample(tinyW, d, Ec, Eu, B, gh, gw, 2, s, seed, trace=trace)
+    assert np.allclose(got, x2, rtol=0, atol=1e-12)
+    assert [(t, c) for t, c, _, _ in trace] == [(1.0, True), (1.0, False), (0.5, True), (0.5, False)]
+    # stop_after = 1 is the state after the first step of the same two-step grid
+    assert np.allclose(o.sample(tinyW, d, Ec, Eu, B, gh, gw, 2, s, seed, stop_after=1), x1, rtol=0, atol=1e-12)
+
+
+def test_sample_wiring_with_padding_masks(tinyW):
+    """One CFG step with different valid text lengths for the two halves ([blog]
+    "Exploring Text Encoder": padded text tokens are masked): the conditional half
+    must use len_cond and the unconditional half len_uncond."""
+    d = TINY
+    rng = np.random.default_rng(10)
+    gh, gw, B, seed, s = 2, 2, 1, 78, 4.0
+    Ec = rng.standard_normal((B, 3, d.txt_layers, d.txt_dim))
+    Eu = rng.standard_normal((B, 3, d.txt_layers, d.txt_dim))
+    C = d.latent_channels
+    z = o.noise(seed, B * C * 4 * gh * gw).astype(np.float64).reshape(B, C, 2 * gh, 2 * gw)
+
+    def f(E, n):
+        return o.unpatchify(o.forward(tinyW, d, o.patchify(z), gh, gw, E, [1.0] * B, txt_len=n), gh, gw, C)
+
+    c, u = f(Ec, [1]), f(Eu, [3])
+    assert np.linalg.norm(f(Ec, [3]) - c) > 1e-3 * np.linalg.norm(c)   # the mask matters here
+    got = o.sample(tinyW, d, Ec, Eu, B, gh, gw, 1, s, seed, len_cond=[1], len_uncond=[3])
+    assert np.allclose(got, z - (u + s * (c - u)), rtol=0, atol=1e-12)
