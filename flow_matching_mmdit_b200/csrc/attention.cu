@@ -371,7 +371,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int rr = 0; rr < 2; ++rr) {
         const int tok = q0 + x * BQ + rlo + 8 * rr;
         if (tok < N) {
-          const float inv = 1.f / (rr ? l1 : l0);
+          // a row with no attended key (l = 0) writes zeros rather than 0 * inf
+          const float lr = rr ? l1 : l0;
+          const float inv = lr > 0.f ? 1.f / lr : 0.f;
           __nv_bfloat16* dst = tok < n_txt ? out_txt + ((int64_t)b * n_txt + tok) * hid
                                            : out_img + ((int64_t)b * (N - n_txt) + (tok - n_txt)) * hid;
           uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + h * 64 + cq);

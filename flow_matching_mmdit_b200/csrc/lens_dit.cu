@@ -1339,6 +1339,11 @@ lens_status lens_op_attention_masked(const uint16_t* q, const uint16_t* k, const
     }
   }
   if (B < 1 || n_txt < 0 || n_img < 0 || n_txt + n_img < 1) return LENS_ERR_SHAPE;
+  // a batch row with no image token and no valid text token has no key to attend:
+  // its softmax is undefined, so the call is refused
+  if (txt_len && n_img == 0)
+    for (int b = 0; b < B; ++b)
+      if (txt_len[b] == 0) return LENS_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15)
     return LENS_ERR_INVALID_ARG;
   int* err = op_err_ptr();

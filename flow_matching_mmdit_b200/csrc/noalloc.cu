@@ -20,6 +20,8 @@ using namespace lens;
 namespace {
 
 constexpr int kNoAllocMaxT = 64;   // timesteps per call
+// the timesteps travel to the feature kernel in a TimestepList by value
+static_assert(kNoAllocMaxT <= kMaxTimesteps, "TimestepList cannot hold kNoAllocMaxT timesteps");
 // sinusoid features [T, 256] followed by the hidden layer [T, 1536], fp32: 448 KiB.
 // Every GPU that loads the library holds this array until the process exits.
 constexpr size_t kScratchFloats = (size_t)kNoAllocMaxT * (kFreqDim + kHidden);
@@ -31,7 +33,10 @@ float* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the array on the current device.  In host code the array's
 // name is only a host-side stand-in, so the address is looked up once per device
-// (with that device current) and cached.
+// (with that device current) and cached.  With lazy module loading (the CUDA
+// default) this lookup is also what loads the module on that device and reserves
+// the array, so it can fail for lack of device memory: that case is reported as
+// LENS_ERR_OOM, any other failure as LENS_ERR_CUDA.
 lens_status scratch_on_current_device(float** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LENS_ERR_CUDA;
@@ -39,8 +44,12 @@ lens_status scratch_on_current_device(float** out) {
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_scratch_ptr[dev]) {
     float* p = nullptr;
-    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_noalloc_scratch) != cudaSuccess || !p)
-      return LENS_ERR_CUDA;
+    const cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_noalloc_scratch);
+    if (e == cudaErrorMemoryAllocation) {
+      cudaGetLastError();
+      return LENS_ERR_OOM;
+    }
+    if (e != cudaSuccess || !p) return LENS_ERR_CUDA;
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
@@ -53,6 +62,8 @@ extern "C" lens_status lens_op_timestep_embed_noalloc(const float* t, int T, con
                                                       const uint16_t* w2, const float* b2, float* temb,
                                                       void* stream) {
   if (!t || !w1 || !w2 || !temb) return LENS_ERR_INVALID_ARG;
+  // the weight rows are read 16 bytes at a time
+  if ((reinterpret_cast<uintptr_t>(w1) | reinterpret_cast<uintptr_t>(w2)) & 15) return LENS_ERR_INVALID_ARG;
   if (T < 1 || T > kNoAllocMaxT) return LENS_ERR_SHAPE;
   for (int i = 0; i < T; ++i)
     if (!isfinite(t[i])) return LENS_ERR_INVALID_ARG;

@@ -327,7 +327,8 @@ LENS_API lens_status lens_op_attention(const uint16_t* q, const uint16_t* k, con
                               void* stream);
 
 /* lens_op_attention with text padding: text keys at and past txt_len[b] (host int
- * [B], B <= 64; NULL = none) are not attended. */
+ * [B], B <= 64; NULL = none) are not attended.  A batch row left with no key at
+ * all (n_img = 0 and txt_len[b] = 0) has no defined softmax: LENS_ERR_SHAPE. */
 LENS_API lens_status lens_op_attention_masked(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
                                               int n_txt, int n_img, const int* txt_len, uint16_t* out_txt,
                                               uint16_t* out_img, void* stream);
@@ -370,12 +371,17 @@ LENS_API lens_status lens_dit_op_text_input(lens_dit* h, const uint16_t* txt, in
  *   w1    dev bf16 [1536, 256],  b1 dev fp32 [1536] or NULL
  *   w2    dev bf16 [1536, 1536], b2 dev fp32 [1536] or NULL
  *   temb  dev fp32 [T, 1536]
- * The intermediates live in one fixed 448 KiB device array inside the library,
- * which every GPU that loads the library keeps until the process exits.  The first
- * call on a device looks up that array's device address (with the device
- * current); make that first call before any stream capture.  All calls share the
- * array and it keeps the last call's contents (every value is written before it
- * is read), so calls whose GPU work overlaps (e.g. on two streams at once) race.
+ * w1 and w2 must be 16-byte aligned (LENS_ERR_INVALID_ARG otherwise).
+ * The intermediates live in one fixed 448 KiB device array inside the library.
+ * The first call on each device looks up that array's device address with the
+ * device current; under lazy module loading (the CUDA default) that lookup is
+ * also what loads the library's kernels on the device and reserves the array,
+ * an implicit driver allocation that may synchronise and may fail (returned as
+ * LENS_ERR_OOM).  So make the first call on each device during set-up, before
+ * any stream capture; later calls allocate nothing, and the array stays reserved
+ * until the process exits.  All calls share the array and it keeps the last
+ * call's contents (every value is written before it is read), so calls whose GPU
+ * work overlaps (e.g. on two streams at once) race.
  * Calls no cudaMalloc, cudaFree or other allocating routine. */
 LENS_API lens_status lens_op_timestep_embed_noalloc(const float* t, int T, const uint16_t* w1, const float* b1,
                                                     const uint16_t* w2, const float* b2, float* temb,

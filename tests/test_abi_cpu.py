@@ -72,3 +72,15 @@ def test_argument_errors_return_synchronously(lib):
     assert lib.lens_op_euler_cfg(ctypes.c_void_p(16), ctypes.c_void_p(16), None, 0, 0.1, 1.0, None) == 2
     assert lib.lens_op_rmsnorm_modulate(ctypes.c_void_p(16), 0, 1, ctypes.c_void_p(16), ctypes.c_void_p(16), 0,
                                         1e-6, ctypes.c_void_p(16), None) == 2
+
+
+def test_attention_with_no_key_is_refused(lib):
+    """A batch row with no image token and no valid text token has no key to attend,
+    so its softmax is undefined: the masked attention op refuses it (SHAPE) before
+    touching the device.  A row that keeps one text key is accepted as far as the
+    size checks go (it then fails on the misaligned fake pointer, INVALID_ARG)."""
+    P = lambda a: ctypes.c_void_p(a)
+    lens = (ctypes.c_int * 2)(3, 0)
+    assert lib.lens_op_attention_masked(P(16), P(16), P(16), 2, 4, 0, lens, P(16), None, None) == 2
+    lens_ok = (ctypes.c_int * 2)(3, 1)
+    assert lib.lens_op_attention_masked(P(8), P(16), P(16), 2, 4, 0, lens_ok, P(16), None, None) == 1
