@@ -21,8 +21,8 @@ STATUS = {0: "LENS_OK", 1: "LENS_ERR_INVALID_ARG", 2: "LENS_ERR_SHAPE", 3: "LENS
 # every symbol include/lens_dit.h declares
 EXPORTS = [
     "lens_dit_default_config", "lens_dit_create", "lens_dit_destroy", "lens_dit_forward", "lens_sample_euler",
-    "lens_dit_debug_blocks", "lens_dit_sync", "lens_status_string", "lens_op_noise_tokens", "lens_op_patchify",
-    "lens_op_unpatchify", "lens_op_rope_table", "lens_op_rmsnorm_modulate", "lens_op_gemm_bf16",
+    "lens_dit_debug_blocks", "lens_dit_debug_raise_abort", "lens_dit_sync", "lens_status_string",
+    "lens_op_noise_tokens", "lens_op_patchify", "lens_op_unpatchify", "lens_op_rope_table", "lens_op_rmsnorm_modulate", "lens_op_gemm_bf16",
     "lens_op_attention", "lens_op_euler_cfg", "lens_dit_op_timestep", "lens_dit_op_text_input",
     "lens_device_sm_count", "lens_dit_profile_kernel", "lens_dit_profile_read", "lens_dit_launch_count",
     "lens_op_timestep_embed_noalloc", "lens_dit_forward_masked", "lens_sample_euler_masked",
@@ -81,6 +81,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "lens_dit_forward": (I, [P, P, I, I, I, P, I, P, P, P]),
         "lens_sample_euler": (I, [P, P, P, I, I, I, I, I, F, U64, P, P]),
         "lens_dit_debug_blocks": (I, [P, I, I, P, P, I, I, I, I, P, P]),
+        "lens_dit_debug_raise_abort": (I, [P, P]),
         "lens_dit_sync": (I, [P, P]),
         "lens_status_string": (ctypes.c_char_p, [I]),
         "lens_op_noise_tokens": (I, [U64, I, I, I, P, P]),
@@ -292,6 +293,10 @@ def lens_dit_debug_blocks(h: LensDit, first: int, last: int, h_img, h_txt, B: in
     tt = np.ascontiguousarray(np.asarray(t, np.float32))
     _check(load_library().lens_dit_debug_blocks(h.ptr, first, last, _ptr(h_img), _ptr(h_txt), B, grid_h, grid_w,
                                                  n_txt, tt.ctypes.data, _stream(stream)), "lens_dit_debug_blocks")
+
+
+def lens_dit_debug_raise_abort(h: LensDit, stream=None) -> None:
+    _check(load_library().lens_dit_debug_raise_abort(h.ptr, _stream(stream)), "lens_dit_debug_raise_abort")
 
 
 def lens_dit_sync(h: LensDit, stream=None) -> None:

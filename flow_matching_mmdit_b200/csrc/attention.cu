@@ -99,6 +99,7 @@ struct Bars {
   uint64_t p_full[TILES];    // softmax -> MMA: P_X written, O_X rescaled
   uint64_t pv_done[TILES];   // MMA -> softmax: O_X += P_X V finished
   uint64_t stagger;          // tile 0 -> tile 1: tile 0 finished its first exponentials
+  uint64_t drain[2];         // each MMA issuer's own completion after an abort
   uint32_t tmem_slot;
 };
 
@@ -135,6 +136,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&bar.pv_done[x], 1);
     }
     mbar_init(&bar.stagger, 8);
+    mbar_init(&bar.drain[0], 1);
+    mbar_init(&bar.drain[1], 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -171,7 +174,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         last_parity[s] = ph;
       }
       mbar_wait_drain(&bar.q_full, 0);
-      if (!ok)
+      // after an abort the consumers may not have waited for every stage filled here
+      if (!ok || err_raised(err))
         for (int s = 0; s < STAGES; ++s)
           if (issued[s]) mbar_wait_drain(&bar.kv_full[s], last_parity[s]);
     }
@@ -203,6 +207,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!ok) break;
         umma_commit(&bar.kv_empty[s]);
       }
+      if (!ok) umma_drain(&bar.drain[0]);   // no S MMA still runs when TMEM is freed
     }
     __syncwarp();
   } else if (warp == 18) {
@@ -231,6 +236,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!ok) break;
         umma_commit(&bar.kv_empty[s]);
       }
+      if (!ok) umma_drain(&bar.drain[1]);   // no P V MMA still runs when TMEM is freed
     }
     __syncwarp();
   } else {

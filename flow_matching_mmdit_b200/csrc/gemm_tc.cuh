@@ -296,7 +296,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* drain = tempty + 2;          // MMA issuer's own completion after an abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -310,6 +311,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 4);
     }
+    mbar_init(drain, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmA0);
     tma_prefetch_desc(&tmB0);
@@ -362,8 +364,9 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
-      if (!ok) {
-        // leave no copy in flight into this CTA's shared memory
+      if (!ok || err_raised(args.err)) {
+        // leave no copy in flight into this CTA's shared memory (after an abort the
+        // consumers may not have waited for every stage this thread filled)
         for (int s = 0; s < STAGES; ++s)
           if (issued[s]) mbar_wait_drain(&full[s], last_parity[s]);
       }
@@ -381,7 +384,10 @@ __global__ void __launch_bounds__(192, 1)
         const int kblocks = args.p[pi].K / C::BK;
         const uint32_t acc = li & 1;
         const uint32_t use = li >> 1;
-        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) break;
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -404,6 +410,7 @@ __global__ void __launch_bounds__(192, 1)
         if (!ok) break;
         umma_commit(&tfull[acc]);
       }
+      if (!ok) umma_drain(drain);   // no UMMA still writes TMEM or reads a stage when the CTA leaves
     }
     __syncwarp();
   } else {
@@ -473,6 +480,26 @@ __device__ __forceinline__ void decode_tile2(const GemmArgs& a, int t, int bn, i
   n0 = (local / P.tiles_m) * bn;
 }
 
+// Abort path of the CTA-pair producer (leader, one thread): make every stage load
+// either CTA issued land before the pair leaves.  L and R are the stage loads the
+// leader and rank 1 issued, in the same (tile, k block) order; a use the leader
+// armed but rank 1 never filled has its missing bytes counted as arrived, a use
+// rank 1 filled but the leader never armed is armed for rank 1's bytes alone.  A
+// CTA issues use i only once use i - STAGES has been consumed, so every use still
+// outstanding lies in [max(L, R) - STAGES, max(L, R)) and is its stage's last.
+template <int STAGES>
+__device__ __forceinline__ void drain_pair_stages(uint64_t* full, uint32_t stage_bytes, uint32_t L, uint32_t R) {
+  const uint32_t hi = L > R ? L : R;
+  for (uint32_t i = hi > (uint32_t)STAGES ? hi - STAGES : 0; i < hi; ++i) {
+    const uint32_t s = i % STAGES, par = (i / STAGES) & 1;
+    if (i >= L)
+      mbar_expect_tx(&full[s], stage_bytes);
+    else if (i >= R)
+      mbar_complete_tx(&full[s], stage_bytes);
+    mbar_wait_drain(&full[s], par);
+  }
+}
+
 template <int BN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     gemm2_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
@@ -491,7 +518,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* drain = tempty + 2;            // leader's MMA completion after an abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint32_t* peer_issued = tmem_slot + 1;   // leader: stage loads rank 1 issued
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -508,6 +537,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 8);
     }
+    mbar_init(drain, 1);
+    *peer_issued = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA0);
     tma_prefetch_desc(&tmB0);
@@ -531,12 +562,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  uint32_t prod_issued = 0;    // producer thread: stage loads issued
+  bool prod_ok = true;
   if (warp == 0) {
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
-      uint32_t last_parity[STAGES];
-      bool issued[STAGES];
-      for (int s = 0; s < STAGES; ++s) issued[s] = false, last_parity[s] = 0;
       bool ok = true;
       for (int t = pair; t < args.total_tiles && ok; t += npairs) {
         int pi, m0, n0;
@@ -552,18 +582,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           if (rank == 0) mbar_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
           tma_load_2d_pair(sA + stage * C::A_BYTES, mA, &full[stage], kb * C::BK, m0 + 128 * (int)rank);
           tma_load_2d_pair(sB + stage * C::B_BYTES, mB, &full[stage], kb * C::BK, n0 + (BN / 2) * (int)rank);
-          issued[stage] = true;
-          last_parity[stage] = phase;
+          ++prod_issued;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
-      if (!ok && rank == 0) {
-        for (int s = 0; s < STAGES; ++s)
-          if (issued[s]) mbar_wait_drain(&full[s], last_parity[s]);
-      }
+      prod_ok = ok;
+      // the leader reconciles both CTAs' loads if the pair aborts
+      if (rank == 1) st_shared_cluster_u32(mapa_shared(smem_u32(peer_issued), 0), prod_issued);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -578,7 +606,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         const int kblocks = args.p[pi].K / C::BK;
         const uint32_t acc = li & 1;
         const uint32_t use = li >> 1;
-        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) break;
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -601,6 +632,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         if (!ok) break;
         umma_commit_pair(&tfull[acc], 0x3);
       }
+      if (!ok) umma_drain_pair(drain);   // no UMMA of the pair still runs when the pair leaves
     }
     __syncwarp();
   } else {
@@ -631,6 +663,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   }
 
   tc_fence_before();
+  cluster_sync_all();          // every role of both CTAs has left its loop; rank 1's count is in place
+  if (warp == 0 && lane == 0 && rank == 0 && (!prod_ok || err_raised(args.err)))
+    drain_pair_stages<STAGES>(full, C::STAGE_BYTES, prod_issued, *peer_issued);
   cluster_sync_all();          // no MMA, TMA or remote arrive of the pair is still in flight
   if (warp == 1) {
     tc_fence_after();

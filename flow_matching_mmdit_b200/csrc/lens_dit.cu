@@ -961,6 +961,13 @@ void lens_dit_destroy(lens_dit* h) {
   delete h;
 }
 
+lens_status lens_dit_debug_raise_abort(lens_dit* h, void* stream) {
+  if (!h) return LENS_ERR_INVALID_ARG;
+  // the flag is a little-endian int that is otherwise 0: its low byte makes it 1
+  if (cudaMemsetAsync(h->err, 1, 1, (cudaStream_t)stream) != cudaSuccess) return LENS_ERR_CUDA;
+  return LENS_OK;
+}
+
 lens_status lens_dit_sync(lens_dit* h, void* stream) {
   if (!h) return LENS_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;

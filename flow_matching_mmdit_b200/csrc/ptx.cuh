@@ -76,6 +76,17 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
+// The grid-wide abort flag, read without caching.
+__device__ __forceinline__ bool err_raised(const int* err) {
+  return *reinterpret_cast<const volatile int*>(err) != 0;
+}
+
+// Count `bytes` of an armed transaction as arrived without any data: used while
+// draining after an abort, for copies that were never issued.
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -146,6 +157,9 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
+}
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
@@ -237,6 +251,20 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
+}
+
+// After an abort: returns once every UMMA this thread issued has completed (bounded),
+// so the TMEM they write may be freed and the shared memory they read reused.
+// `bar` is a barrier of count 1 used for nothing else.
+__device__ __forceinline__ void umma_drain(uint64_t* bar) {
+  umma_commit(bar);
+  mbar_wait_drain(bar, 0);
+}
+// The same for the leader of a CTA pair (the pair's UMMAs write both CTAs' TMEM);
+// the commit arrives on the leader's `bar` only.
+__device__ __forceinline__ void umma_drain_pair(uint64_t* bar) {
+  umma_commit_pair(bar, 0x1);
+  mbar_wait_drain(bar, 0);
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 D, both K-major.

@@ -167,7 +167,8 @@ __global__ void __launch_bounds__(kW4Threads, 1)
   uint64_t* empty = bfull + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* drain = tempty + 2;          // MMA issuer's own completion after an abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -182,6 +183,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 4);
     }
+    mbar_init(drain, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmX0);
     tma_prefetch_desc(&tmQ0);
@@ -245,7 +247,8 @@ __global__ void __launch_bounds__(kW4Threads, 1)
           }
         }
       }
-      if (!ok) {
+      if (!ok || err_raised(args.err)) {
+        // after an abort the consumers may not have waited for every stage filled here
         for (int s = 0; s < STAGES; ++s)
           if (issued[s]) mbar_wait_drain(&full[s], last_parity[s]);
       }
@@ -263,7 +266,10 @@ __global__ void __launch_bounds__(kW4Threads, 1)
         const int kblocks = args.p[pi].K / C::BK;
         const uint32_t acc = li & 1;
         const uint32_t use = li >> 1;
-        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) break;
+        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * MH * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
@@ -289,6 +295,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
         if (!ok) break;
         umma_commit(&tfull[acc]);
       }
+      if (!ok) umma_drain(drain);   // no UMMA still writes TMEM or reads a stage when the CTA leaves
     }
     __syncwarp();
   } else if (warp < 6) {

@@ -254,6 +254,13 @@ LENS_API lens_status lens_dit_debug_blocks(lens_dit* h, int first, int last, flo
                                   int B, int grid_h, int grid_w, int n_txt, const float* t,
                                   void* stream);
 
+/* Test hook for the failure path: raise the handle's device abort flag on `stream`,
+ * as an expired wait would.  Kernels launched after it leave at their first wait
+ * that does not complete at once, after draining their own copies and MMAs; the
+ * next lens_dit_sync reports LENS_ERR_TIMEOUT and clears the flag, and calls after
+ * that run normally.  Errors: INVALID_ARG (NULL handle), CUDA. */
+LENS_API lens_status lens_dit_debug_raise_abort(lens_dit* h, void* stream);
+
 /* Wait for the handle's work on `stream` and report kernel-side errors
  * (CUDA errors, TIMEOUT from the device watchdog).  Clears the watchdog flag. */
 LENS_API lens_status lens_dit_sync(lens_dit* h, void* stream);

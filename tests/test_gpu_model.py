@@ -422,3 +422,32 @@ def test_step_sampler_state_rules(small):
         L.lens_sampler_update(h, 0, v, None)
     assert e.value.status == 1
     _sync(h)
+
+
+# ------------------------------------------------------------------ failure path (no fault: a flag the test raises)
+@pytest.mark.parametrize("gh,gw,nt", [(8, 8, 16), (32, 32, 128)])
+def test_abort_flag_reports_timeout_then_recovers(small, gh, gw, nt):
+    """With the device abort flag raised (as an expired wait would raise it) every
+    kernel that waits leaves at its first wait that does not complete at once, after
+    draining its own TMA copies and MMAs; lens_dit_sync reports LENS_ERR_TIMEOUT (5)
+    and clears the flag, and the next forward matches the oracle again.  Nothing
+    faults or hangs: the flag is the designed abort path."""
+    d, w, h = small
+    B = 2
+    X = image_tokens(B, gh * gw, 31)
+    E = text_features(B, nt, 32)
+    t = [0.6, 0.2]
+    v = torch.empty((B, gh * gw, 128), dtype=torch.float32, device="cuda")
+    L.lens_dit_debug_raise_abort(h)
+    L.lens_dit_forward(h, dev(X), B, gh, gw, dev(E), nt, t, v)
+    with pytest.raises(L.LensError) as e:
+        L.lens_dit_sync(h)
+    assert e.value.status == 5
+    _sync(h)                                         # the flag was cleared
+    v.fill_(float("nan"))
+    L.lens_dit_forward(h, dev(X), B, gh, gw, dev(E), nt, t, v)
+    _sync(h)
+    ref = o.forward(o.Weights(w), d, X, gh, gw, E, t)
+    got = host(v)
+    assert np.all(np.isfinite(got))
+    assert cos_sim(got, ref) > 0.9999 and rel_l2(got, ref) < 1e-2
