@@ -160,6 +160,27 @@ def job_value(units_per_step_per_rank: float, n_ranks: int, ms_per_step: float) 
     return n_ranks * units_per_step_per_rank / (ms_per_step / 1e3)
 
 
+# ---------------------------------------------------------------- CFG split over rank pairs
+def cfg_split_error(wl, gpus: int, world: int):
+    """Why --cfg-split cannot run with these settings (None when it can)."""
+    if wl.guidance == 1.0:
+        return "--cfg-split needs a CFG workload (guidance != 1)"
+    if gpus < 2 or gpus % 2 or world != gpus:
+        return "--cfg-split needs an even --gpus >= 2, launched as that many torchrun ranks"
+    return None
+
+
+def cfg_split_plan(wl, rank: int, world: int) -> dict:
+    """This rank's part of a CFG-split job: pair p = rank // 2 samples seed wl.seed +
+    1000 p; half 0 runs the conditional text (features drawn from that seed), half 1 the
+    unconditional (zeros).  units_per_rank: image tokens through the denoiser per step
+    and rank, so that job_value over all ranks counts each pair's sample once."""
+    pair, half = rank // 2, rank % 2
+    seed = wl.seed + 1000 * pair
+    return {"pair": pair, "half": half, "pairs": world // 2, "seed": seed, "text_seed": seed,
+            "conditional": half == 0, "units_per_rank": wl.batch * wl.n_img * wl.steps / 2.0}
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -251,7 +272,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="turbo_1024", choices=[k for k, v in WORKLOADS.items() if v.steps > 0])
+    ap.add_argument("--workload", default=None, choices=[k for k, v in WORKLOADS.items() if v.steps > 0],
+                    help="default: turbo_1024 (cfg_1024 with --cfg-split)")
     ap.add_argument("--impl", default="lens", choices=["lens", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cfg-rescale", type=float, default=0.0,
@@ -262,16 +284,29 @@ def main():
                     help="valid text tokens per sample (the rest are padding, masked in attention)")
     ap.add_argument("--weight-bits", type=int, default=16, choices=[16, 4],
                     help="4: int4 weight-only block Linears (group 64), quantized at create")
+    ap.add_argument("--cfg-split", action="store_true",
+                    help="CFG halves on rank pairs (even --gpus >= 2 under torchrun): the conditional and the "
+                         "unconditional forward of each sample on two GPUs, one velocity all-gather per step")
     args = ap.parse_args()
+    if args.workload is None:
+        args.workload = "cfg_1024" if args.cfg_split else "turbo_1024"
     wl = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.cfg_split:
+        err = cfg_split_error(wl, args.gpus, world)
+        if err:
+            print(json.dumps({"metric": METRIC, "error": err}), flush=True)
+            return 2
     config = {"workload": f"{args.workload}: {wl.name}", "batch": wl.batch, "img_tokens": wl.n_img,
               "txt_tokens": wl.n_txt, "sampling_steps": wl.steps, "guidance": wl.guidance, "blocks": 48,
               "forward_rows": wl.batch * (2 if wl.guidance != 1.0 else 1),
               "l2": "inputs larger than L2: 8.2 GB of weights streamed by every forward",
               "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+    if args.cfg_split:
+        config["forward_rows"] = wl.batch            # each rank runs one half of the CFG batch
+        config["parallelism"] = f"CFG split: {world // 2} rank pair(s), one velocity all-gather per step"
     if args.txt_valid is not None:
         config["txt_valid"] = args.txt_valid
     if args.weight_bits != 16:
@@ -309,7 +344,8 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
     cfg.weight_bits = args.weight_bits
     h = L.lens_dit_create(cfg, weights)
     del weights
-    seed = wl.seed + 1000 * rank
+    plan = cfg_split_plan(wl, rank, world) if args.cfg_split else None
+    seed = plan["seed"] if plan else wl.seed + 1000 * rank
     txt_host = text_features(wl.batch, wl.n_txt, seed)
     txt = torch.from_numpy(txt_host.view(np.int16)).cuda()
     out = torch.empty((wl.batch, 32, 2 * wl.grid_h, 2 * wl.grid_w), dtype=torch.float32, device="cuda")
@@ -322,9 +358,18 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
 
     lens = None if args.txt_valid is None else [args.txt_valid] * wl.batch
 
-    def sample(text):
-        L.lens_sample_euler_ex(h, text, lens, None, lens, wl.batch, wl.n_txt, wl.height_px, wl.width_px, wl.steps,
-                               opt, seed, out)
+    if plan:
+        from flow_matching_mmdit_b200 import cfg_split
+        groups = cfg_split.pair_groups(world, dist.new_group)
+
+        def sample(text):
+            cfg_split.sample_cfg_split(h, text if plan["conditional"] else None, lens, wl.batch, wl.n_txt,
+                                       wl.height_px, wl.width_px, wl.steps, opt, seed, out, groups[plan["pair"]],
+                                       plan["half"])
+    else:
+        def sample(text):
+            L.lens_sample_euler_ex(h, text, lens, None, lens, wl.batch, wl.n_txt, wl.height_px, wl.width_px,
+                                   wl.steps, opt, seed, out)
 
     def step():
         sample(txt)
@@ -388,7 +433,7 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
     ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], dist, "cuda")
 
     ms_step = ms_total / args.steps
-    tokens_per_step = wl.batch * wl.n_img * wl.steps
+    tokens_per_step = plan["units_per_rank"] if plan else wl.batch * wl.n_img * wl.steps
     value = job_value(tokens_per_step, args.gpus, ms_step)
     e2e_value = job_value(tokens_per_step, args.gpus, e2e_ms / args.steps)
     flops_step = wl.steps * config["forward_rows"] * forward_flops(wl.n_img, wl.n_txt)

@@ -7,9 +7,16 @@
 // output accumulate in TMEM, the running row max and sum live in registers of the
 // softmax warps, base-2 exponentials carry the 1/8 scale.  Keys past N are masked;
 // rows past N are computed on zero-filled queries and never stored.
+#include "exp2_poly.h"
 #include "gemm.h"
 #include "kernels.cuh"
 #include "smem_attr.h"
+
+// Which of each thread's 16 groups of four scores per key tile take their
+// exponentials on the FMA pipe (bit g set) instead of the exponential unit.
+#ifndef LENS_ATTN_EMU_MASK
+#define LENS_ATTN_EMU_MASK 0x0000u
+#endif
 
 namespace lens {
 
@@ -42,6 +49,30 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x0, 2^x1 of a packed pair on the FMA pipe: exp2_poly (exp2_poly.h) step by step
+// on fp32 pairs, with the clamp and the exponent add on the integer side.
+__device__ __forceinline__ void exp2_fma_pair(uint64_t x, float& a, float& b) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, kExp2Floor), fmaxf(x1, kExp2Floor));
+  const uint64_t t = f2_add(xc, f2_pack(kExp2Round, kExp2Round));
+  const uint64_t f = f2_sub(xc, f2_sub(t, f2_pack(kExp2Round, kExp2Round)));
+  uint64_t p = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  a = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  b = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 // three-input maximum (one instruction on sm_100)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
@@ -318,10 +349,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t pk[32];
 #pragma unroll
       for (int g = 0; g < 16; ++g) {
-        float x0, x1, x2, x3;
-        f2_unpack(f2_fma(f2_pack(sc[4 * g], sc[4 * g + 1]), sl2, nb0), x0, x1);
-        f2_unpack(f2_fma(f2_pack(sc[4 * g + 2], sc[4 * g + 3]), sl2, nb1), x2, x3);
-        const float e0 = ex2(x0), e1 = ex2(x1), e2 = ex2(x2), e3 = ex2(x3);
+        const uint64_t x01 = f2_fma(f2_pack(sc[4 * g], sc[4 * g + 1]), sl2, nb0);
+        const uint64_t x23 = f2_fma(f2_pack(sc[4 * g + 2], sc[4 * g + 3]), sl2, nb1);
+        float e0, e1, e2, e3;
+        if ((LENS_ATTN_EMU_MASK >> g) & 1u) {
+          exp2_fma_pair(x01, e0, e1);
+          exp2_fma_pair(x23, e2, e3);
+        } else {
+          float x0, x1, x2, x3;
+          f2_unpack(x01, x0, x1);
+          f2_unpack(x23, x2, x3);
+          e0 = ex2(x0);
+          e1 = ex2(x1);
+          e2 = ex2(x2);
+          e3 = ex2(x3);
+        }
         a0[g & 1] = f2_add(a0[g & 1], f2_pack(e0, e1));
         a1[g & 1] = f2_add(a1[g & 1], f2_pack(e2, e3));
         pk[2 * g] = pack_bf16x2(e0, e1);

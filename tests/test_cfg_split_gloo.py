@@ -95,3 +95,82 @@ def test_pairing_rules():
     for bad in (1, 3):
         with pytest.raises(ValueError):
             cfg_split.pair_groups(bad, lambda r: None)
+
+
+# ------------------------------------------------------------------ bench.py --cfg-split plumbing
+def test_bench_cfg_split_plan_and_refusals():
+    import bench
+    from lens_inputs import WORKLOADS
+    wl = WORKLOADS["cfg_1024"]
+    plans = [bench.cfg_split_plan(wl, r, 4) for r in range(4)]
+    assert [(p["pair"], p["half"], p["conditional"]) for p in plans] == \
+        [(0, 0, True), (0, 1, False), (1, 0, True), (1, 1, False)]
+    assert plans[0]["seed"] == plans[1]["seed"] != plans[2]["seed"] == plans[3]["seed"]
+    # whole-job units: each pair's sample counted once
+    total = sum(p["units_per_rank"] for p in plans)
+    assert total == 2 * wl.batch * wl.n_img * wl.steps
+    assert bench.job_value(plans[0]["units_per_rank"], 4, 1000.0) == pytest.approx(total)
+    assert bench.cfg_split_error(wl, 2, 2) is None
+    assert bench.cfg_split_error(wl, 1, 1) and bench.cfg_split_error(wl, 3, 3) and bench.cfg_split_error(wl, 4, 2)
+    assert bench.cfg_split_error(WORKLOADS["turbo_1024"], 2, 2)
+
+
+class _WallTimer:
+    def start(self):
+        import time
+        self.t0 = time.perf_counter()
+
+    def stop(self):
+        import time
+        self.t1 = time.perf_counter()
+
+    def elapsed_ms(self):
+        return (self.t1 - self.t0) * 1e3
+
+
+def _bench_worker(rank, world, port, q):
+    import bench
+    from lens_inputs import WORKLOADS
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        plan = bench.cfg_split_plan(WORKLOADS["cfg_1024"], rank, world)
+        groups = cfg_split.pair_groups(world, dist.new_group)
+        W = o.Weights(make_weights(TINY, seed=11, std=0.2, bias_std=0.05, gain_std=0.2))
+        Ec = text_features(B, NT, plan["text_seed"], TINY)
+        E = Ec if plan["conditional"] else np.zeros_like(Ec)
+        runs = []
+
+        def step():
+            ops = OracleSteps(W, E, plan["seed"], None, 0.0)
+            cfg_split.cfg_split_steps(ops, STEPS, plan["half"], cfg_split.make_gather(groups[plan["pair"]],
+                                                                                     dist.all_gather))
+            runs.append(ops.x)
+
+        ms = bench.timed_region(step, 2, dist.barrier, lambda: None, _WallTimer())
+        mx = bench.max_over_ranks([ms], dist, "cpu")
+        q.put((rank, runs, mx, plan["seed"], plan["text_seed"]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_cfg_split_timed_steps_on_two_ranks():
+    """The two ranks of one pair, timed the way bench.py --cfg-split times them: exactly
+    K steps each, both halves end on the same latent, equal to the batched sampler."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_bench_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict((r[0], r[1:]) for r in (q.get(timeout=300) for _ in range(world)))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (runs0, mx0, seed, tseed), (runs1, mx1, _, _) = res[0], res[1]
+    assert len(runs0) == len(runs1) == 2 and mx0 == mx1
+    W = o.Weights(make_weights(TINY, seed=11, std=0.2, bias_std=0.05, gain_std=0.2))
+    ref = o.sample(W, TINY, text_features(B, NT, tseed, TINY), None, B, GH, GW, STEPS, G, seed)
+    for a, b in zip(runs0, runs1):
+        assert np.array_equal(a, b)
+        assert np.allclose(a, ref, rtol=0, atol=1e-10)
