@@ -2,6 +2,9 @@
 
     python -m flow_matching_mmdit_b200.build [--force] [--verbose]
 
+LENS_NVCC_EXTRA (environment) adds nvcc flags to every compile, e.g.
+LENS_NVCC_EXTRA="-DLENS_ATTN_EMU_MASK=0x5555u" for a measurement build (use --force).
+
 Objects go to flow_matching_mmdit_b200/_build/; the shared library is written next
 to this file so it travels with the source tree.  The CUDA runtime is linked
 statically and the driver API is reached through cudaGetDriverEntryPoint, so the
@@ -53,7 +56,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
         obj = os.path.join(BUILD, src.replace(".cu", ".o"))
         objs.append(obj)
         if force or _stale(obj, deps):
-            cmd = [nvcc()] + ARCH + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + [
+            extra = os.environ.get("LENS_NVCC_EXTRA", "").split()
+            cmd = [nvcc()] + ARCH + FLAGS + extra + (["-Xptxas", "-v"] if ptxas_verbose else []) + [
                 "-c", os.path.join(CSRC, src), "-o", obj]
             if verbose:
                 print(" ".join(cmd), flush=True)
