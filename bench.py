@@ -37,7 +37,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from lens_inputs import LENS, WORKLOADS, make_weights, text_features  # noqa: E402
+from lens_inputs import LENS, WORKLOADS, image_tokens, make_weights, text_features  # noqa: E402
 
 METRIC = "DiT img-tokens/s per 1024² forward; ms per 4-step 1024² sample; % bf16 peak"
 SPEC_BF16_TFLOPS = 2250.0
@@ -272,8 +272,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default=None, choices=[k for k, v in WORKLOADS.items() if v.steps > 0],
-                    help="default: turbo_1024 (cfg_1024 with --cfg-split)")
+    ap.add_argument("--workload", default=None, choices=[k for k, v in WORKLOADS.items() if v.num_blocks == 48],
+                    help="default: turbo_1024 (cfg_1024 with --cfg-split); fwd_512 times single forwards")
     ap.add_argument("--impl", default="lens", choices=["lens", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cfg-rescale", type=float, default=0.0,
@@ -362,12 +362,21 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
         from flow_matching_mmdit_b200 import cfg_split
         groups = cfg_split.pair_groups(world, dist.new_group)
 
-        def sample(text):
+        def sample(text):                            # noqa: F811
             cfg_split.sample_cfg_split(h, text if plan["conditional"] else None, lens, wl.batch, wl.n_txt,
                                        wl.height_px, wl.width_px, wl.steps, opt, seed, out, groups[plan["pair"]],
                                        plan["half"])
+    elif wl.steps == 0:
+        # a single-forward workload: one step = one 48-block forward of seeded N(0, 1) tokens at wl.t
+        tok_host = image_tokens(wl.batch, wl.n_img, seed)
+        tok = torch.from_numpy(tok_host).cuda()
+        out = torch.empty((wl.batch, wl.n_img, 128), dtype=torch.float32, device="cuda")
+
+        def sample(text):                            # noqa: F811
+            L.lens_dit_forward_masked(h, tok, wl.batch, wl.grid_h, wl.grid_w, text, wl.n_txt, lens,
+                                      [wl.t] * wl.batch, out)
     else:
-        def sample(text):
+        def sample(text):                            # noqa: F811
             L.lens_sample_euler_ex(h, text, lens, None, lens, wl.batch, wl.n_txt, wl.height_px, wl.width_px,
                                    wl.steps, opt, seed, out)
 
@@ -422,8 +431,12 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
         sample(txt_dev)
         out_pinned.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
+    tok_pinned = torch.from_numpy(tok_host).pin_memory() if wl.steps == 0 else None
+
     def e2e_step():
         txt_dev.copy_(txt_pinned, non_blocking=True)
+        if tok_pinned is not None:
+            tok.copy_(tok_pinned, non_blocking=True)
         sample(txt_dev)
         out_pinned.copy_(out, non_blocking=True)
 
@@ -433,10 +446,11 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
     ms_total, e2e_ms = max_over_ranks([ms_total, e2e_ms], dist, "cuda")
 
     ms_step = ms_total / args.steps
-    tokens_per_step = plan["units_per_rank"] if plan else wl.batch * wl.n_img * wl.steps
+    forwards = max(wl.steps, 1)
+    tokens_per_step = plan["units_per_rank"] if plan else wl.batch * wl.n_img * forwards
     value = job_value(tokens_per_step, args.gpus, ms_step)
     e2e_value = job_value(tokens_per_step, args.gpus, e2e_ms / args.steps)
-    flops_step = wl.steps * config["forward_rows"] * forward_flops(wl.n_img, wl.n_txt)
+    flops_step = forwards * config["forward_rows"] * forward_flops(wl.n_img, wl.n_txt)
     peaks = measured_peaks()
     tflops = flops_step / (ms_step / 1e3) / 1e12
 
@@ -472,7 +486,8 @@ def _run_lens(args, wl, config, world, rank, local, torch, L):
                           f"of_{peaks['source']}_burst": round(tflops * 1e0 / peaks["bf16_tflops"], 4),
                           f"of_{peaks['source']}_sustained": round(tflops / peaks["bf16_tflops_sustained"], 4)},
         "e2e": {"value": round(e2e_value, 1), "unit": "img-tokens/s",
-                "h2d_bytes_per_step": int(txt_host.nbytes), "d2h_bytes_per_step": int(out.numel() * 4),
+                "h2d_bytes_per_step": int(txt_host.nbytes) + (int(tok_host.nbytes) if wl.steps == 0 else 0),
+                "d2h_bytes_per_step": int(out.numel() * 4),
                 "ms_per_step": round(e2e_ms / args.steps, 3)},
         "roofline": roof, "gpu_launches": int(gpu_launches), "clocks": clk.summary(),
         "context": {"pages_h100_turbo_4step_1024_s": 0.84, "pages_h100_20step_cfg5_1024_s": 3.15,

@@ -182,6 +182,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar.tmem_slot;
+  grid_dependency_sync();    // set-up above touched only shared memory and TMEM
 
   if (warp == 16) {
     // ---------------------------------------------------------------- TMA producer
@@ -466,9 +467,8 @@ cudaError_t launch_joint_attention(const __nv_bfloat16* q, const __nv_bfloat16* 
   }
   dim3 grid((N + tc::TILES * tc::BQ - 1) / (tc::TILES * tc::BQ), heads, B);
   const float scale_log2 = 0.125f * 1.4426950408889634f;
-  tc::joint_attention_tc_kernel<<<grid, tc::THREADS, tc::SMEM, st>>>(tq, tk, tv, N, n_txt, heads, out_txt, out_img,
-                                                                        scale_log2, lens, err);
-  return cudaGetLastError();
+  return launch_pdl(tc::joint_attention_tc_kernel, grid, dim3(tc::THREADS), tc::SMEM, st, tq, tk, tv, N, n_txt, heads,
+                    out_txt, out_img, scale_log2, lens, err);
 }
 
 }  // namespace lens

@@ -124,37 +124,66 @@ __global__ void rope_table_kernel(int gh, int gw, int n_txt, int ntok, float2* _
 // One warp per row of 1536 fp32: y = (1 + scale) * x * rsqrt(mean(x^2) + eps) + shift.
 // Up to two independent segments (the image and the text stream of a block) share
 // one launch: rows [0, s0.M) belong to segment 0, the next s1.M rows to segment 1.
+// Every warp issues its row's twelve 16-byte loads first; meanwhile the CTA stages
+// the shift and 1 + scale of its first row's sample in shared memory once (12 KB),
+// so the eight warps of a CTA read them from there instead of each pulling them
+// through L1.  A warp whose row belongs to another sample or segment (a CTA that
+// straddles a boundary) reads its own from global memory.
 // 64 registers (4 blocks of 256 per SM): the 4352 rows of a 1024^2 block fit one wave.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ const RmsSeg* rms_row_segment(const RmsSeg& s0, const RmsSeg& s1, int& row) {
+  if (row < s0.M) return &s0;
+  row -= s0.M;
+  return row < s1.M ? &s1 : nullptr;
+}
+
 __global__ void __launch_bounds__(256, 4) rmsnorm_modulate_kernel(RmsSeg s0, RmsSeg s1, float eps) {
+  __shared__ float4 sm_shift[kHidden / 4], sm_scale[kHidden / 4];
+  grid_dependency_sync();
+  // the CTA's first row decides which sample's modulation is staged; the copies are
+  // asynchronous (global -> shared, no registers) and overlap the row loads below
+  int row0 = blockIdx.x * (blockDim.x >> 5);
+  const RmsSeg* sg0 = rms_row_segment(s0, s1, row0);       // never null: the grid covers M rows
+  const int b0 = row0 / sg0->rows_per_batch;
+  for (int i = threadIdx.x; i < kHidden / 4; i += blockDim.x) {
+    cp_async16(&sm_shift[i], sg0->shift + b0 * sg0->mod_stride + 4 * i);
+    cp_async16(&sm_scale[i], sg0->scale + b0 * sg0->mod_stride + 4 * i);
+  }
+  cp_async_commit();
   int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  const RmsSeg* sg = &s0;
-  if (row >= s0.M) {
-    row -= s0.M;
-    sg = &s1;
-    if (row >= s1.M) return;
-  }
-  const float4* xr = reinterpret_cast<const float4*>(sg->x + (int64_t)row * kHidden);
+  const RmsSeg* sg = rms_row_segment(s0, s1, row);
   float4 v[12];
+  if (sg) {
+    const float4* xr = reinterpret_cast<const float4*>(sg->x + (int64_t)row * kHidden);
+#pragma unroll
+    for (int i = 0; i < 12; ++i) v[i] = xr[lane + 32 * i];
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  if (!sg) return;
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < 12; ++i) {
-    v[i] = xr[lane + 32 * i];
-    ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
-  }
+  for (int i = 0; i < 12; ++i) ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float r = rsqrtf(ss * (1.0f / kHidden) + eps);
   const int b = row / sg->rows_per_batch;
-  const float4* sh = reinterpret_cast<const float4*>(sg->shift + b * sg->mod_stride);
-  const float4* sc = reinterpret_cast<const float4*>(sg->scale + b * sg->mod_stride);
+  const bool staged = sg == sg0 && b == b0;
+  const float4* sh = staged ? sm_shift : reinterpret_cast<const float4*>(sg->shift + b * sg->mod_stride);
+  const float4* sc = staged ? sm_scale : reinterpret_cast<const float4*>(sg->scale + b * sg->mod_stride);
   uint2* yr = reinterpret_cast<uint2*>(sg->y + (int64_t)row * kHidden);
 #pragma unroll
   for (int i = 0; i < 12; ++i) {
-    const float4 a = __ldg(sh + lane + 32 * i), s = __ldg(sc + lane + 32 * i);
+    const float4 a = sh[lane + 32 * i], c = sc[lane + 32 * i];
     uint2 w;
-    w.x = pack_bf16x2((1.f + s.x) * v[i].x * r + a.x, (1.f + s.y) * v[i].y * r + a.y);
-    w.y = pack_bf16x2((1.f + s.z) * v[i].z * r + a.z, (1.f + s.w) * v[i].w * r + a.w);
+    w.x = pack_bf16x2((1.f + c.x) * v[i].x * r + a.x, (1.f + c.y) * v[i].y * r + a.y);
+    w.y = pack_bf16x2((1.f + c.z) * v[i].z * r + a.z, (1.f + c.w) * v[i].w * r + a.w);
     yr[lane + 32 * i] = w;
   }
 }
@@ -336,8 +365,7 @@ cudaError_t launch_rope_table(int gh, int gw, int n_txt, float2* table, cudaStre
 cudaError_t launch_rmsnorm_modulate(const RmsSeg& s0, const RmsSeg& s1, float eps, cudaStream_t st) {
   const int M = s0.M + s1.M;
   if (M <= 0) return cudaSuccess;
-  rmsnorm_modulate_kernel<<<(M + 7) / 8, 256, 0, st>>>(s0, s1, eps);
-  return cudaGetLastError();
+  return launch_pdl(rmsnorm_modulate_kernel, dim3((M + 7) / 8), dim3(256), 0, st, s0, s1, eps);
 }
 cudaError_t launch_rmsnorm_modulate(const float* x, int M, int rows_per_batch, const float* shift,
                                     const float* scale, int64_t mod_stride, float eps, __nv_bfloat16* y,

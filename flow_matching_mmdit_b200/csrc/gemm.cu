@@ -36,8 +36,7 @@ cudaError_t launch_one(const CUtensorMap& A0, const CUtensorMap& B0, const CUten
     if (e != cudaSuccess) return e;
   }
   const int grid = args.total_tiles < sms ? args.total_tiles : sms;
-  gemm_tc_kernel<BN, EPI><<<grid, 192, C::SMEM, st>>>(A0, B0, A1, B1, C0, C1, args);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(192), C::SMEM, st, A0, B0, A1, B1, C0, C1, args);
 }
 
 template <int BN, int EPI>
@@ -51,8 +50,8 @@ cudaError_t launch_pair(const CUtensorMap& A0, const CUtensorMap& B0, const CUte
     if (e != cudaSuccess) return e;
   }
   const int pairs = args.total_tiles < sms / 2 ? args.total_tiles : sms / 2;
-  gemm2_tc_kernel<BN, EPI><<<2 * pairs, 192, C::SMEM, st>>>(A0, B0, A1, B1, C0, C1, args);
-  return cudaGetLastError();
+  return launch_pdl(gemm2_tc_kernel<BN, EPI>, dim3(2 * pairs), dim3(192), C::SMEM, st, A0, B0, A1, B1, C0, C1,
+                    args);
 }
 
 }  // namespace

@@ -334,6 +334,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dependency_sync();    // set-up above touched only shared memory, TMEM and weights
 
   if (warp == 0) {
     if (lane == 0) {
@@ -561,6 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   cluster_sync_all();          // both CTAs' barriers initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dependency_sync();      // set-up above touched only shared memory, TMEM and weights
 
   uint32_t prod_issued = 0;    // producer thread: stage loads issued
   bool prod_ok = true;

@@ -15,6 +15,7 @@
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
 #include "lens_dit.h"
+#include "smem_attr.h"
 
 using namespace lens;
 
@@ -147,20 +148,35 @@ static const char* kStatusStr[] = {"ok", "invalid argument", "shape out of range
   } while (0)
 
 // Launch accounting: count every kernel, and time the selected family.
+// One event record of the profiling hooks.  While the stream is being captured the
+// record must be an external one to become an event node of the graph; outside a
+// capture it is a plain record.  A failed record is cleared so that it is not
+// reported as the next launch's error.
+static bool prof_record(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  const cudaError_t e = cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal)
+                                                            : cudaEventRecord(ev, st);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e == cudaSuccess;
+}
+
 struct KScope {
   lens_dit* h;
   cudaStream_t st;
   bool on;
   KScope(lens_dit* h_, int kind, cudaStream_t st_) : h(h_), st(st_), on(false) {
     ++h->launches;
-    if (h->prof_kind == kind && h->prof_n < h->prof_cap) {
-      // external records become real event nodes when the stream is being captured
-      on = cudaEventRecordWithFlags(h->prof_ev[2 * h->prof_n], st, cudaEventRecordExternal) == cudaSuccess;
-    }
+    if (h->prof_kind == kind && h->prof_n < h->prof_cap) on = prof_record(h->prof_ev[2 * h->prof_n], st);
+    // a timed launch sits between two event records: no programmatic overlap with it
+    pdl_suspended() = on;
   }
   ~KScope() {
-    if (on && cudaEventRecordWithFlags(h->prof_ev[2 * h->prof_n + 1], st, cudaEventRecordExternal) == cudaSuccess)
-      ++h->prof_n;
+    pdl_suspended() = false;
+    if (on && prof_record(h->prof_ev[2 * h->prof_n + 1], st)) ++h->prof_n;
   }
 };
 
