@@ -50,8 +50,8 @@ cudaError_t launch_pair(const CUtensorMap& A0, const CUtensorMap& B0, const CUte
     if (e != cudaSuccess) return e;
   }
   const int pairs = args.total_tiles < sms / 2 ? args.total_tiles : sms / 2;
-  return launch_pdl(gemm2_tc_kernel<BN, EPI>, dim3(2 * pairs), dim3(192), C::SMEM, st, A0, B0, A1, B1, C0, C1,
-                    args);
+  return launch_pdl(gemm2_tc_kernel<BN, EPI>, dim3(2 * pairs), dim3(C::THREADS), C::SMEM, st, A0, B0, A1, B1, C0,
+                    C1, args);
 }
 
 }  // namespace

@@ -90,16 +90,18 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, int t, int bn, in
   n0 = (local / P.tiles_m) * bn;
 }
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+// SiLU with the fast reciprocal division (the result is rounded to bf16): for very
+// negative x the denominator overflows to inf and the quotient is 0, the limit.
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 // ------------------------------------------------------------------ epilogues
 // Stage one 32-row x 128-byte box (this thread's row = `lane`) in the warp's next
 // shared-memory slot with the 128-byte swizzle, then let lane 0 ship it.
-template <bool REDUCE>
+template <bool REDUCE, int NSLOTS>
 __device__ __forceinline__ void stage_and_ship(uint8_t* slots, uint32_t& slot, const uint4 (&chunk)[8],
                                                const CUtensorMap* map, int x, int y, bool ship) {
   const int lane = threadIdx.x & 31;
-  if (lane == 0) bulk_wait_read<1>();          // the slot's previous box has been read out
+  if (lane == 0) bulk_wait_read<NSLOTS - 1>();   // the slot's previous box has been read out
   __syncwarp();
   uint8_t* buf = slots + slot * 4096;
 #pragma unroll
@@ -114,23 +116,43 @@ __device__ __forceinline__ void stage_and_ship(uint8_t* slots, uint32_t& slot, c
       tma_store_2d(map, buf, x, y);
   }
   if (lane == 0) bulk_commit();
-  slot ^= 1;
+  if (NSLOTS == 2) slot ^= 1;
 }
 
-template <int BN, int EPI>
+// `part` of `parts` column ranges of the tile (32-column chunks, SwiGLU 128-column
+// groups, QKV heads) is this warp's; the other parts go to warps reading the same
+// TMEM lanes.  NSLOTS staging slots of 4 KB per warp.
+template <int BN, int EPI, int NSLOTS = 2>
 __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtensorMap* tmC, int row, int row0_warp,
                                               int n0, uint32_t taddr, uint8_t* slots, uint32_t& slot,
-                                              const float* qk_gains) {
+                                              const float* qk_gains, int part = 0, int parts = 1) {
   const bool live = row < P.M;
   const bool any_live = row0_warp < P.M;
   if constexpr (EPI == EPI_F32 || EPI == EPI_RESID) {
     const float* gate = nullptr;
+    const int c_begin = part * (BN / 32) / parts, c_end = (part + 1) * (BN / 32) / parts;
+    float4 gnext[8];                     // the gates of the next chunk, loaded one chunk ahead
     if constexpr (EPI == EPI_RESID) {
       const int b = live ? row / P.rows_per_batch : 0;
       gate = P.gate + (int64_t)b * P.gate_stride + n0;
+      if (live) {
+        const float4* g4 = reinterpret_cast<const float4*>(gate + c_begin * 32);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) gnext[j] = __ldg(g4 + j);
+      }
     }
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = c_begin; c < c_end; ++c) {
+      float4 gcur[8];
+      if constexpr (EPI == EPI_RESID) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) gcur[j] = gnext[j];
+        if (live && c + 1 < c_end) {
+          const float4* g4 = reinterpret_cast<const float4*>(gate + (c + 1) * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) gnext[j] = __ldg(g4 + j);
+        }
+      }
       float r[32];
       tmem_ld32(taddr + c * 32, r);
       tmem_ld_wait();
@@ -141,14 +163,12 @@ __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtens
       }
       if constexpr (EPI == EPI_RESID) {
         if (live) {
-          const float4* g4 = reinterpret_cast<const float4*>(gate + col);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float4 g = __ldg(g4 + j);
-            r[4 * j] *= g.x;
-            r[4 * j + 1] *= g.y;
-            r[4 * j + 2] *= g.z;
-            r[4 * j + 3] *= g.w;
+            r[4 * j] *= gcur[j].x;
+            r[4 * j + 1] *= gcur[j].y;
+            r[4 * j + 2] *= gcur[j].z;
+            r[4 * j + 3] *= gcur[j].w;
           }
         }
       }
@@ -157,13 +177,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtens
       for (int j = 0; j < 8; ++j)
         ch[j] = make_uint4(__float_as_uint(r[4 * j]), __float_as_uint(r[4 * j + 1]), __float_as_uint(r[4 * j + 2]),
                            __float_as_uint(r[4 * j + 3]));
-      stage_and_ship<EPI == EPI_RESID>(slots, slot, ch, tmC, n0 + col, row0_warp, any_live);
+      stage_and_ship<EPI == EPI_RESID, NSLOTS>(slots, slot, ch, tmC, n0 + col, row0_warp, any_live);
     }
   } else if constexpr (EPI == EPI_SWIGLU) {
     // B rows were packed [w1 rows 32c..32c+31 | w3 rows 32c..32c+31] per 64 columns;
     // every 128 accumulator columns give 64 outputs = one 128-byte box row
 #pragma unroll 1
-    for (int c = 0; c < BN / 128; ++c) {
+    for (int c = part * (BN / 128) / parts; c < (part + 1) * (BN / 128) / parts; ++c) {
       uint4 ch[8];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -187,7 +207,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtens
                          pack_bf16x2(silu_f(g[8 * j + 4]) * u[8 * j + 4], silu_f(g[8 * j + 5]) * u[8 * j + 5]),
                          pack_bf16x2(silu_f(g[8 * j + 6]) * u[8 * j + 6], silu_f(g[8 * j + 7]) * u[8 * j + 7]));
       }
-      stage_and_ship<false>(slots, slot, ch, tmC, n0 / 2 + c * 64, row0_warp, any_live);
+      stage_and_ship<false, NSLOTS>(slots, slot, ch, tmC, n0 / 2 + c * 64, row0_warp, any_live);
     }
   } else if constexpr (EPI == EPI_QKV) {
     // gains: the problem's q and k gains staged in shared memory at kernel start
@@ -205,7 +225,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtens
       for (int p = 0; p < 16; ++p) rp[p] = __ldg(rope4 + p);
     }
 #pragma unroll 1
-    for (int hh = 0; hh < BN / 64; ++hh) {
+    for (int hh = part * (BN / 64) / parts; hh < (part + 1) * (BN / 64) / parts; ++hh) {
       float x[64];
       tmem_ld32(taddr + hh * 64, *reinterpret_cast<float(*)[32]>(&x[0]));
       tmem_ld32(taddr + hh * 64 + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
@@ -435,7 +455,9 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
     if constexpr (epi_uses_tma(EPI)) {
-      if (lane == 0) bulk_wait<0>();           // every box has landed before the CTA leaves
+      // every box has been read out of shared memory before the CTA leaves; the
+      // grid's completion covers the writes to global memory
+      if (lane == 0) bulk_wait_read<0>();
       __syncwarp();
     }
   }
@@ -457,15 +479,26 @@ __global__ void __launch_bounds__(192, 1)
 //   full[s]    (leader)  TMA bytes of both CTAs; armed by the leader's producer
 //   empty[s]   (both)    MMA commit multicast: stage s may be refilled
 //   tfull[a]   (both)    MMA commit multicast: accumulator a holds a finished tile
-//   tempty[a]  (leader)  8 arrivals (4 epilogue warps x 2 CTAs): accumulator a free
+//   tempty[a]  (leader)  2 x epilogue warps arrivals (both CTAs): accumulator a free
+// The SwiGLU epilogue (a SiLU per output) runs on eight warps per CTA (320 threads),
+// two per TMEM lane quarter, each taking half of a tile's 128-column groups: on four
+// it took longer than the next tile's main loop (measured 23 % of the launch at the
+// 1024^2 shape), and the MMA waited for a free accumulator.  One 4 KB staging slot
+// each, the same 32 KB as four warps with two.  The other epilogues keep four warps:
+// the residual ones are bound by the TMA reduce-add, and the QKV one measured slower
+// on eight (three heads split 2 / 1, more warps beside the MMA issuer).
 template <int BN, int EPI>
 struct Gemm2Cfg {
   static constexpr int BM = 128, BK = 64;
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = (BN / 2) * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_WARPS = EPI == EPI_SWIGLU ? 8 : 4;
+  static constexpr int EPI_PARTS = EPI_WARPS / 4;            // column parts per TMEM lane quarter
+  static constexpr int EPI_SLOTS = 2 / EPI_PARTS;            // 4 KB staging slots per epilogue warp
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr uint32_t EPI_SLOT = 4096;
-  static constexpr uint32_t EPI_BYTES = epi_uses_tma(EPI) ? 4 * 2 * EPI_SLOT : 0;
+  static constexpr uint32_t EPI_BYTES = epi_uses_tma(EPI) ? EPI_WARPS * EPI_SLOTS * EPI_SLOT : 0;
   static constexpr uint32_t AUX_BYTES = EPI == EPI_QKV ? 1024 : 0;
   static constexpr uint32_t BUDGET = 232448 - 1024 - 256 - EPI_BYTES - AUX_BYTES;
   static constexpr int STAGES = (BUDGET / STAGE_BYTES) > 8 ? 8 : (BUDGET / STAGE_BYTES);
@@ -502,7 +535,7 @@ __device__ __forceinline__ void drain_pair_stages(uint64_t* full, uint32_t stage
 }
 
 template <int BN, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::THREADS, 1)
     gemm2_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                     const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1,
@@ -536,7 +569,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 8);
+      mbar_init(&tempty[a], 2 * C::EPI_WARPS);
     }
     mbar_init(drain, 1);
     *peer_issued = 0;
@@ -638,8 +671,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    const int quarter = warp & 3;
-    uint8_t* slots = sEpi + quarter * 2 * C::EPI_SLOT;
+    const int quarter = warp & 3;                 // TMEM lanes 32 quarter .. + 31
+    const int part = (warp - 2) >> 2;             // which part of the tile's columns
+    uint8_t* slots = sEpi + (warp - 2) * C::EPI_SLOTS * C::EPI_SLOT;
     uint32_t slot = 0;
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
     int li = 0;
@@ -652,14 +686,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       tc_fence_after();
       const int row0 = m0 + 128 * (int)rank + quarter * 32;
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
-      epilogue_tile<BN, EPI>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots, slot,
-                             sAux + pi * 128);
+      epilogue_tile<BN, EPI, C::EPI_SLOTS>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots,
+                                           slot, sAux + pi * 128, part, C::EPI_PARTS);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + acc * 8);
     }
-    if constexpr (epi_uses_tma(EPI)) {
-      if (lane == 0) bulk_wait<0>();
+    if constexpr (C::EPI_BYTES > 0) {
+      if (lane == 0) bulk_wait_read<0>();      // as above
       __syncwarp();
     }
   }

@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kW4Threads, 1)
       if (lane == 0) mbar_arrive(&tempty[acc]);
     }
     if constexpr (epi_uses_tma(EPI)) {
-      if (lane == 0) bulk_wait<0>();
+      if (lane == 0) bulk_wait_read<0>();      // read out of shared memory; the grid covers the rest
       __syncwarp();
     }
   } else {
