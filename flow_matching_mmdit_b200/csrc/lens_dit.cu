@@ -28,7 +28,7 @@ constexpr size_t kStageElems = (size_t)kModPerStream * kHidden;
 // 128 wide for w1|w3 and QKV, 96 wide for the 1536-wide to_out and w2 (272 tiles)
 constexpr int kBnW13W4 = 128, kBnQkvW4 = 128, kBnResW4 = 96;
 
-constexpr int kBnQkv = 192, kBnOut = 192, kBnW13 = 256, kBnW2 = 192, kBnImgIn = 256, kBnTxtIn = 128,
+constexpr int kBnQkv = 256, kBnOut = 192, kBnW13 = 256, kBnW2 = 192, kBnImgIn = 256, kBnTxtIn = 128,
               kBnProj = 128;
 
 // a 4-bit weight (weight_bits = 4): codes and scales in lens_op_quantize_w4's layout
