@@ -43,7 +43,7 @@ METRIC = "DiT img-tokens/s per 1024² forward; ms per 4-step 1024² sample; % bf
 SPEC_BF16_TFLOPS = 2250.0
 KERNEL_FAMILIES = ["attention", "gemm_qkv", "gemm_out", "gemm_w13", "gemm_w2", "rmsnorm_mod", "gemm_mod"]
 KERNEL_SOURCES = {
-    "attention": ["attention.cu"],
+    "attention": ["attention.cu", "ptx.cuh", "exp2_poly.h"],
     "gemm_qkv": ["gemm_tc.cuh", "gemm.cu", "ptx.cuh"], "gemm_out": ["gemm_tc.cuh", "gemm.cu", "ptx.cuh"],
     "gemm_w13": ["gemm_tc.cuh", "gemm.cu", "ptx.cuh"], "gemm_w2": ["gemm_tc.cuh", "gemm.cu", "ptx.cuh"],
     "gemm_mod": ["gemm_tc.cuh", "gemm.cu", "ptx.cuh"], "rmsnorm_mod": ["elementwise.cu"],

@@ -136,10 +136,27 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-__device__ __forceinline__ const RmsSeg* rms_row_segment(const RmsSeg& s0, const RmsSeg& s1, int& row) {
-  if (row < s0.M) return &s0;
-  row -= s0.M;
-  return row < s1.M ? &s1 : nullptr;
+// The row's segment, picked field by field: taking the address of a by-value kernel
+// parameter would make the compiler copy both segments to local memory.
+struct RmsRow {
+  const float* x;
+  const float* shift;
+  const float* scale;
+  __nv_bfloat16* y;
+  bool ok;
+};
+__device__ __forceinline__ RmsRow rms_row(const RmsSeg& s0, const RmsSeg& s1, int row) {
+  const bool second = row >= s0.M;
+  const int r = second ? row - s0.M : row;
+  const int b = r / (second ? s1.rows_per_batch : s0.rows_per_batch);
+  const int64_t mod = b * (second ? s1.mod_stride : s0.mod_stride);
+  RmsRow o;
+  o.ok = !second || r < s1.M;
+  o.x = (second ? s1.x : s0.x) + (int64_t)r * kHidden;
+  o.y = (second ? s1.y : s0.y) + (int64_t)r * kHidden;
+  o.shift = (second ? s1.shift : s0.shift) + mod;
+  o.scale = (second ? s1.scale : s0.scale) + mod;
+  return o;
 }
 
 __global__ void __launch_bounds__(256, 4) rmsnorm_modulate_kernel(RmsSeg s0, RmsSeg s1, float eps) {
@@ -147,37 +164,33 @@ __global__ void __launch_bounds__(256, 4) rmsnorm_modulate_kernel(RmsSeg s0, Rms
   grid_dependency_sync();
   // the CTA's first row decides which sample's modulation is staged; the copies are
   // asynchronous (global -> shared, no registers) and overlap the row loads below
-  int row0 = blockIdx.x * (blockDim.x >> 5);
-  const RmsSeg* sg0 = rms_row_segment(s0, s1, row0);       // never null: the grid covers M rows
-  const int b0 = row0 / sg0->rows_per_batch;
+  const RmsRow first = rms_row(s0, s1, blockIdx.x * (blockDim.x >> 5));   // ok: the grid covers M rows
   for (int i = threadIdx.x; i < kHidden / 4; i += blockDim.x) {
-    cp_async16(&sm_shift[i], sg0->shift + b0 * sg0->mod_stride + 4 * i);
-    cp_async16(&sm_scale[i], sg0->scale + b0 * sg0->mod_stride + 4 * i);
+    cp_async16(&sm_shift[i], first.shift + 4 * i);
+    cp_async16(&sm_scale[i], first.scale + 4 * i);
   }
   cp_async_commit();
-  int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const RmsRow rw = rms_row(s0, s1, blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5));
   const int lane = threadIdx.x & 31;
-  const RmsSeg* sg = rms_row_segment(s0, s1, row);
   float4 v[12];
-  if (sg) {
-    const float4* xr = reinterpret_cast<const float4*>(sg->x + (int64_t)row * kHidden);
+  if (rw.ok) {
+    const float4* xr = reinterpret_cast<const float4*>(rw.x);
 #pragma unroll
     for (int i = 0; i < 12; ++i) v[i] = xr[lane + 32 * i];
   }
   cp_async_wait_all();
   __syncthreads();
-  if (!sg) return;
+  if (!rw.ok) return;
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < 12; ++i) ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float r = rsqrtf(ss * (1.0f / kHidden) + eps);
-  const int b = row / sg->rows_per_batch;
-  const bool staged = sg == sg0 && b == b0;
-  const float4* sh = staged ? sm_shift : reinterpret_cast<const float4*>(sg->shift + b * sg->mod_stride);
-  const float4* sc = staged ? sm_scale : reinterpret_cast<const float4*>(sg->scale + b * sg->mod_stride);
-  uint2* yr = reinterpret_cast<uint2*>(sg->y + (int64_t)row * kHidden);
+  const bool staged = rw.shift == first.shift;
+  const float4* sh = staged ? sm_shift : reinterpret_cast<const float4*>(rw.shift);
+  const float4* sc = staged ? sm_scale : reinterpret_cast<const float4*>(rw.scale);
+  uint2* yr = reinterpret_cast<uint2*>(rw.y);
 #pragma unroll
   for (int i = 0; i < 12; ++i) {
     const float4 a = sh[lane + 32 * i], c = sc[lane + 32 * i];

@@ -7,8 +7,9 @@ profiling (ncu) and quick timing:
 `attention` runs the joint-attention op on random q, k, v of the workload's
 sequence; `blocks` runs `blocks` denoiser blocks (every GEMM epilogue, attention and
 RMSNorm) through the debug hook of a model with that many blocks; `gemm` runs the
-plain tcgen05 GEMM op at M = rows x tokens, N = 8192, K = 1536.  Prints the
-CUDA-event time per iteration.
+plain tcgen05 GEMM op at M = rows x tokens, N = 8192, K = 1536; `rmsnorm` runs
+RMSNorm + modulate over all rows x tokens fp32 rows (one sample's shift and scale
+per batch row).  Prints the CUDA-event time per iteration.
 """
 from __future__ import annotations
 
@@ -30,7 +31,7 @@ def main() -> int:
     from lens_inputs import LENS, WORKLOADS, f32_to_bf16_bits, make_weights
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", choices=["attention", "blocks", "gemm"], required=True)
+    ap.add_argument("--case", choices=["attention", "blocks", "gemm", "rmsnorm"], required=True)
     ap.add_argument("--workload", default="turbo_1024")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--blocks", type=int, default=2)
@@ -40,6 +41,7 @@ def main() -> int:
     N = wl.n_img + wl.n_txt
     rng = np.random.default_rng(0)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    unit = "TFLOP/s"
 
     if a.case == "attention":
         q, k, v = (torch.from_numpy(f32_to_bf16_bits(rng.standard_normal((rows, 24, N, 64)).astype(np.float32))
@@ -56,6 +58,13 @@ def main() -> int:
         C = torch.empty((M, 8192), dtype=torch.float32, device="cuda")
         run = lambda: L.lens_op_gemm_bf16(A, B, None, C, M, 8192, 1536)
         flops = 2.0 * M * 8192 * 1536
+    elif a.case == "rmsnorm":
+        M = rows * N
+        x = torch.from_numpy(rng.standard_normal((M, 1536)).astype(np.float32) * 3).cuda()
+        mod = torch.from_numpy(rng.standard_normal((rows, 6 * 1536)).astype(np.float32) * 0.2).cuda()
+        y = torch.empty((M, 1536), dtype=torch.int16, device="cuda")
+        run = lambda: L.lens_op_rmsnorm_modulate(x, M, N, mod[:, 1536:], mod[:, 3072:], 6 * 1536, 1e-6, y)
+        flops, unit = M * 1536 * 6.0, "TB/s"   # bytes: fp32 in, bf16 out
     else:
         d = LENS.with_blocks(a.blocks)
         cfg = L.lens_dit_default_config()
@@ -76,7 +85,7 @@ def main() -> int:
         ev1.record()
         torch.cuda.synchronize()
         ms = ev0.elapsed_time(ev1)
-        print(f"{a.case} {a.workload} iter {i}: {ms:.3f} ms, {flops / ms / 1e9:.1f} TFLOP/s", flush=True)
+        print(f"{a.case} {a.workload} iter {i}: {ms:.3f} ms, {flops / ms / 1e9:.2f} {unit}", flush=True)
     return 0
 
 
