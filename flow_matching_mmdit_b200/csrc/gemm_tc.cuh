@@ -119,13 +119,40 @@ __device__ __forceinline__ void stage_and_ship(uint8_t* slots, uint32_t& slot, c
   if (NSLOTS == 2) slot ^= 1;
 }
 
+// Per-row operands of a tile's epilogue that do not depend on the accumulator, loaded
+// before the wait for it so that their latency hides behind that wait: the gates of the
+// first 32-column chunk of this warp's part (residual epilogue, pre[0..7]), or this
+// row's RoPE (cos, sin) pairs (QKV epilogue on a q or k tile, pre[0..15]).
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_prefetch(const GemmProblem& P, int row, int n0, int part, int parts,
+                                                  float4 (&pre)[16]) {
+  if (row >= P.M) return;
+  const int b = row / P.rows_per_batch;
+  if constexpr (EPI == EPI_RESID) {
+    const float4* g4 = reinterpret_cast<const float4*>(P.gate + (int64_t)b * P.gate_stride + n0 +
+                                                       part * (BN / 32) / parts * 32);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) pre[j] = __ldg(g4 + j);
+  } else if constexpr (EPI == EPI_QKV) {
+    if (n0 / (P.heads * 64) < 2) {
+      const int tok = P.tok_offset + row - b * P.rows_per_batch;
+      const float4* rope4 = reinterpret_cast<const float4*>(P.rope + (int64_t)tok * 32);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) pre[j] = __ldg(rope4 + j);
+    }
+  }
+}
+
 // `part` of `parts` column ranges of the tile (32-column chunks, SwiGLU 128-column
 // groups, QKV heads) is this warp's; the other parts go to warps reading the same
-// TMEM lanes.  NSLOTS staging slots of 4 KB per warp.
-template <int BN, int EPI, int NSLOTS = 2>
+// TMEM lanes.  NSLOTS staging slots of 4 KB per warp.  With PRE, `pre` holds what
+// epilogue_prefetch loaded for this tile (the residual and QKV epilogues use it);
+// without, the epilogue loads those operands itself.
+template <int BN, int EPI, int NSLOTS = 2, bool PRE = true>
 __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtensorMap* tmC, int row, int row0_warp,
                                               int n0, uint32_t taddr, uint8_t* slots, uint32_t& slot,
-                                              const float* qk_gains, int part = 0, int parts = 1) {
+                                              const float* qk_gains, const float4 (&pre)[16], int part = 0,
+                                              int parts = 1) {
   const bool live = row < P.M;
   const bool any_live = row0_warp < P.M;
   if constexpr (EPI == EPI_F32 || EPI == EPI_RESID) {
@@ -138,7 +165,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtens
       if (live) {
         const float4* g4 = reinterpret_cast<const float4*>(gate + c_begin * 32);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) gnext[j] = __ldg(g4 + j);
+        for (int j = 0; j < 8; ++j) gnext[j] = PRE ? pre[j] : __ldg(g4 + j);
       }
     }
 #pragma unroll 1
@@ -218,12 +245,15 @@ __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtens
     const int tok = P.tok_offset + (live ? row - b * P.rows_per_batch : 0);
     __nv_bfloat16* base = sec == 0 ? P.q : (sec == 1 ? P.k : P.v);
     const float4* gain4 = reinterpret_cast<const float4*>(qk_gains + (sec == 0 ? 0 : 64));
-    float4 rp[16];                                // this row's (cos, sin) pairs, once per tile
-    if (sec < 2 && live) {
-      const float4* rope4 = reinterpret_cast<const float4*>(P.rope + (int64_t)tok * 32);
+    float4 rown[16];
+    if constexpr (!PRE) {
+      if (sec < 2 && live) {
+        const float4* rope4 = reinterpret_cast<const float4*>(P.rope + (int64_t)tok * 32);
 #pragma unroll
-      for (int p = 0; p < 16; ++p) rp[p] = __ldg(rope4 + p);
+        for (int p = 0; p < 16; ++p) rown[p] = __ldg(rope4 + p);
+      }
     }
+    const float4 (&rp)[16] = *(PRE ? &pre : &rown);   // this row's (cos, sin) pairs (q and k tiles)
 #pragma unroll 1
     for (int hh = part * (BN / 64) / parts; hh < (part + 1) * (BN / 64) / parts; ++hh) {
       float x[64];
@@ -444,12 +474,14 @@ __global__ void __launch_bounds__(192, 1)
       decode_tile(args, t, BN, pi, m0, n0);
       const uint32_t acc = li & 1;
       const uint32_t use = li >> 1;
+      const int row0 = m0 + quarter * 32;
+      float4 pre[16];
+      epilogue_prefetch<BN, EPI>(args.p[pi], row0 + lane, n0, 0, 1, pre);
       if (!mbar_wait(&tfull[acc], use & 1, args.err)) break;
       tc_fence_after();
-      const int row0 = m0 + quarter * 32;
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
       epilogue_tile<BN, EPI>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots, slot,
-                             sAux + pi * 128);
+                             sAux + pi * 128, pre);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -682,12 +714,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
       decode_tile2(args, t, BN, pi, m0, n0);
       const uint32_t acc = li & 1;
       const uint32_t use = li >> 1;
+      const int row0 = m0 + 128 * (int)rank + quarter * 32;
+      float4 pre[16];
+      epilogue_prefetch<BN, EPI>(args.p[pi], row0 + lane, n0, part, C::EPI_PARTS, pre);
       if (!mbar_wait(&tfull[acc], use & 1, args.err)) break;
       tc_fence_after();
-      const int row0 = m0 + 128 * (int)rank + quarter * 32;
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
       epilogue_tile<BN, EPI, C::EPI_SLOTS>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots,
-                                           slot, sAux + pi * 128, part, C::EPI_PARTS);
+                                           slot, sAux + pi * 128, pre, part, C::EPI_PARTS);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + acc * 8);

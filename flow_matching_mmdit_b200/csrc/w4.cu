@@ -314,8 +314,9 @@ __global__ void __launch_bounds__(kW4Threads, 1)
       for (int h = 0; h < MH; ++h) {
         const int row0 = m0 + 128 * h + quarter * 32;
         const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * MH * BN + h * BN;
-        epilogue_tile<BN, EPI>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots, slot,
-                               sAux + pi * 128);
+        const float4 none[16] = {};   // the epilogue loads its per-row operands itself here
+        epilogue_tile<BN, EPI, 2, false>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots,
+                                         slot, sAux + pi * 128, none);
       }
       tc_fence_before();
       __syncwarp();
