@@ -134,6 +134,8 @@ struct Bars {
   uint32_t tmem_slot;
 };
 
+static_assert(sizeof(Bars) <= 256, "barriers overflow their shared-memory reserve");
+
 __global__ void __launch_bounds__(THREADS, 1)
     joint_attention_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                               const __grid_constant__ CUtensorMap tmV, int N, int n_txt, int heads,
