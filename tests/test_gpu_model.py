@@ -397,6 +397,13 @@ def test_cfg_split_halves_reproduce_the_fused_sampler(small, gh, gw, nt, steps, 
         _sync(h)
         assert np.array_equal(host(outs[0]), host(outs[1]))
         assert np.array_equal(host(outs[0]), host(ref))
+        if gh * gw <= 64:
+            # and against the oracle's sampler (affordable at this size)
+            mu64 = None if mu is None else float(np.float32(mu))
+            want = o.sample(o.Weights(w), d, text_features(B, nt, 61), None, B, gh, gw, steps, 5.0, seed, mu=mu64,
+                            phi=phi)
+            got = host(outs[0])
+            assert cos_sim(got, want) >= 0.99 and rel_l2(got, want) <= 5e-2, (cos_sim(got, want), rel_l2(got, want))
     finally:
         h2.destroy()
 
