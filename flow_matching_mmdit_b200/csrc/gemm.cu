@@ -39,10 +39,35 @@ cudaError_t launch_one(const CUtensorMap& A0, const CUtensorMap& B0, const CUten
   return launch_pdl(gemm_tc_kernel<BN, EPI>, dim3(grid), dim3(192), C::SMEM, st, A0, B0, A1, B1, C0, C1, args);
 }
 
+// Tail of a CTA-pair launch: the last round of whole tiles (T mod pairs of them) would
+// leave the other pairs idle for a whole tile time.  Split each of those tiles into s
+// column slices (s = 4 or 2, the largest whose slices all fit in one round, whose
+// width the MMA (multiple of 16) and the epilogue's unit allow: 32 columns for the
+// fp32 and residual epilogues, a 64-column head for QKV, a 128-column w1|w3 group for
+// SwiGLU, and for which narrow B maps were given).  Every output element is still one
+// MMA chain over the whole K.  Returns the index into NarrowB (-1: no split).
+static int plan_tail(GemmArgs& a, int pairs, int bn, int epi, const NarrowB* nb) {
+  const int rounds = a.total_tiles / pairs;
+  const int tail = a.total_tiles - rounds * pairs;
+  if (!nb || rounds < 1 || tail == 0) return -1;
+  const int unit = epi == EPI_SWIGLU ? 128 : (epi == EPI_QKV ? 64 : 32);
+  for (int i = 1; i >= 0; --i) {
+    const int s = 2 << i;
+    const int w = bn / s;
+    if (bn % s || w % unit || w % 16 || tail * s > pairs) continue;
+    if (!nb->b0[i] || (a.num_problems > 1 && !nb->b1[i])) continue;
+    a.tail_begin = rounds * pairs;
+    a.tail_split = s;
+    a.total_items = a.tail_begin + tail * s;
+    return i;
+  }
+  return -1;
+}
+
 template <int BN, int EPI>
 cudaError_t launch_pair(const CUtensorMap& A0, const CUtensorMap& B0, const CUtensorMap& A1, const CUtensorMap& B1,
                         const CUtensorMap& C0, const CUtensorMap& C1, const GemmArgs& args, int sms,
-                        cudaStream_t st) {
+                        cudaStream_t st, const NarrowB* nb) {
   using C = Gemm2Cfg<BN, EPI>;
   static std::atomic<uint64_t> attr{0};
   {
@@ -50,8 +75,12 @@ cudaError_t launch_pair(const CUtensorMap& A0, const CUtensorMap& B0, const CUte
     if (e != cudaSuccess) return e;
   }
   const int pairs = args.total_tiles < sms / 2 ? args.total_tiles : sms / 2;
+  GemmArgs a = args;
+  const int n = plan_tail(a, pairs, BN, EPI, nb);
+  const CUtensorMap& B0n = n >= 0 ? *nb->b0[n] : B0;
+  const CUtensorMap& B1n = n >= 0 && a.num_problems > 1 ? *nb->b1[n] : B0n;
   return launch_pdl(gemm2_tc_kernel<BN, EPI>, dim3(2 * pairs), dim3(C::THREADS), C::SMEM, st, A0, B0, A1, B1, C0,
-                    C1, args);
+                    C1, B0n, B1n, a);
 }
 
 }  // namespace
@@ -137,6 +166,9 @@ void finalize_problems(GemmArgs& a, int bn, int bm) {
     begin += p.tiles_m * p.tiles_n;
   }
   a.total_tiles = begin;
+  a.tail_begin = begin;
+  a.tail_split = 1;
+  a.total_items = begin;
 }
 
 cudaError_t launch_gemm(int bn, int epi, const CUtensorMap* A0, const CUtensorMap* B0, const CUtensorMap* A1,
@@ -172,7 +204,7 @@ cudaError_t launch_gemm(int bn, int epi, const CUtensorMap* A0, const CUtensorMa
 
 cudaError_t launch_gemm_pair(int bn, int epi, const CUtensorMap* A0, const CUtensorMap* B0, const CUtensorMap* A1,
                              const CUtensorMap* B1, const CUtensorMap* C0, const CUtensorMap* C1, GemmArgs& args,
-                             int sms, cudaStream_t st) {
+                             int sms, cudaStream_t st, const NarrowB* narrow) {
   finalize_problems(args, bn, 256);
   if (args.total_tiles == 0) return cudaSuccess;
   if ((epi == EPI_F32 || epi == EPI_RESID || epi == EPI_SWIGLU) && (!C0 || (args.num_problems > 1 && !C1)))
@@ -182,7 +214,7 @@ cudaError_t launch_gemm_pair(int bn, int epi, const CUtensorMap* A0, const CUten
   const CUtensorMap& c0 = C0 ? *C0 : *A0;
   const CUtensorMap& c1 = C1 ? *C1 : c0;
 #define LENS_GEMM2_CASE(BN_, EPI_) \
-  if (bn == BN_ && epi == EPI_) return launch_pair<BN_, EPI_>(*A0, *B0, a1, b1, c0, c1, args, sms, st);
+  if (bn == BN_ && epi == EPI_) return launch_pair<BN_, EPI_>(*A0, *B0, a1, b1, c0, c1, args, sms, st, narrow);
   LENS_GEMM2_CASE(256, EPI_F32)
   LENS_GEMM2_CASE(128, EPI_F32)
   LENS_GEMM2_CASE(192, EPI_RESID)

@@ -62,10 +62,19 @@ cudaError_t launch_gemm(int bn, int epi, const CUtensorMap* A0, const CUtensorMa
                         const CUtensorMap* B1, const CUtensorMap* C0, const CUtensorMap* C1, GemmArgs& args, int sms,
                         cudaStream_t st);
 
+// B maps of the same weights with boxes of bn / 4 and bn / 8 rows (index 0 and 1):
+// the tail items of a pair launch cut into 2 or 4 column slices load only their own
+// rows through them.  A null entry rules that split out.
+struct NarrowB {
+  const CUtensorMap* b0[2];
+  const CUtensorMap* b1[2];
+};
+
 // The same on 256 x bn tiles computed by CTA pairs (cta_group::2): A maps keep a box
 // of 128 rows, B maps need a box of bn / 2 rows.  Grid = 2 x min(tiles, sms / 2).
+// With `narrow`, the last, partly filled round of tiles may run as column slices.
 cudaError_t launch_gemm_pair(int bn, int epi, const CUtensorMap* A0, const CUtensorMap* B0, const CUtensorMap* A1,
                              const CUtensorMap* B1, const CUtensorMap* C0, const CUtensorMap* C1, GemmArgs& args,
-                             int sms, cudaStream_t st);
+                             int sms, cudaStream_t st, const NarrowB* narrow = nullptr);
 
 }  // namespace lens

@@ -56,6 +56,12 @@ struct GemmArgs {
   GemmProblem p[2];
   int num_problems;
   int total_tiles;
+  // CTA-pair kernel: tiles [tail_begin, total_tiles) (the last, partly filled round)
+  // are each computed as tail_split narrower tiles of BN / tail_split columns, so that
+  // they spread over the CTA pairs that would otherwise idle; total_items counts
+  // the work items that result.  The other kernels leave them at (total_tiles, 1,
+  // total_tiles).
+  int tail_begin, tail_split, total_items;
   int* err;
 };
 
@@ -125,12 +131,12 @@ __device__ __forceinline__ void stage_and_ship(uint8_t* slots, uint32_t& slot, c
 // row's RoPE (cos, sin) pairs (QKV epilogue on a q or k tile, pre[0..15]).
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_prefetch(const GemmProblem& P, int row, int n0, int part, int parts,
-                                                  float4 (&pre)[16]) {
+                                                  float4 (&pre)[16], int width = BN) {
   if (row >= P.M) return;
   const int b = row / P.rows_per_batch;
   if constexpr (EPI == EPI_RESID) {
     const float4* g4 = reinterpret_cast<const float4*>(P.gate + (int64_t)b * P.gate_stride + n0 +
-                                                       part * (BN / 32) / parts * 32);
+                                                       part * (width / 32) / parts * 32);
 #pragma unroll
     for (int j = 0; j < 8; ++j) pre[j] = __ldg(g4 + j);
   } else if constexpr (EPI == EPI_QKV) {
@@ -152,12 +158,12 @@ template <int BN, int EPI, int NSLOTS = 2, bool PRE = true>
 __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtensorMap* tmC, int row, int row0_warp,
                                               int n0, uint32_t taddr, uint8_t* slots, uint32_t& slot,
                                               const float* qk_gains, const float4 (&pre)[16], int part = 0,
-                                              int parts = 1) {
+                                              int parts = 1, int width = BN) {
   const bool live = row < P.M;
   const bool any_live = row0_warp < P.M;
   if constexpr (EPI == EPI_F32 || EPI == EPI_RESID) {
     const float* gate = nullptr;
-    const int c_begin = part * (BN / 32) / parts, c_end = (part + 1) * (BN / 32) / parts;
+    const int c_begin = part * (width / 32) / parts, c_end = (part + 1) * (width / 32) / parts;
     float4 gnext[8];                     // the gates of the next chunk, loaded one chunk ahead
     if constexpr (EPI == EPI_RESID) {
       const int b = live ? row / P.rows_per_batch : 0;
@@ -210,7 +216,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtens
     // B rows were packed [w1 rows 32c..32c+31 | w3 rows 32c..32c+31] per 64 columns;
     // every 128 accumulator columns give 64 outputs = one 128-byte box row
 #pragma unroll 1
-    for (int c = part * (BN / 128) / parts; c < (part + 1) * (BN / 128) / parts; ++c) {
+    for (int c = part * (width / 128) / parts; c < (part + 1) * (width / 128) / parts; ++c) {
       uint4 ch[8];
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -255,7 +261,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmProblem& P, const CUtens
     }
     const float4 (&rp)[16] = *(PRE ? &pre : &rown);   // this row's (cos, sin) pairs (q and k tiles)
 #pragma unroll 1
-    for (int hh = part * (BN / 64) / parts; hh < (part + 1) * (BN / 64) / parts; ++hh) {
+    for (int hh = part * (width / 64) / parts; hh < (part + 1) * (width / 64) / parts; ++hh) {
       float x[64];
       tmem_ld32(taddr + hh * 64, *reinterpret_cast<float(*)[32]>(&x[0]));
       tmem_ld32(taddr + hh * 64 + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
@@ -546,6 +552,23 @@ __device__ __forceinline__ void decode_tile2(const GemmArgs& a, int t, int bn, i
   n0 = (local / P.tiles_m) * bn;
 }
 
+// Work item w: a whole tile, or one of the tail_split column slices of a tail tile.
+// Each output element is still one MMA chain over the whole K, so its value does
+// not depend on which kind of item computed it.
+__device__ __forceinline__ void decode_item2(const GemmArgs& a, int w, int bn, int& pi, int& m0, int& n0,
+                                             int& width) {
+  int t = w, sub = 0;
+  width = bn;
+  if (w >= a.tail_begin) {
+    const int q = w - a.tail_begin;
+    t = a.tail_begin + q / a.tail_split;
+    sub = q - (q / a.tail_split) * a.tail_split;
+    width = bn / a.tail_split;
+  }
+  decode_tile2(a, t, bn, pi, m0, n0);
+  n0 += sub * width;
+}
+
 // Abort path of the CTA-pair producer (leader, one thread): make every stage load
 // either CTA issued land before the pair leaves.  L and R are the stage loads the
 // leader and rank 1 issued, in the same (tile, k block) order; a use the leader
@@ -553,17 +576,30 @@ __device__ __forceinline__ void decode_tile2(const GemmArgs& a, int t, int bn, i
 // rank 1 filled but the leader never armed is armed for rank 1's bytes alone.  A
 // CTA issues use i only once use i - STAGES has been consumed, so every use still
 // outstanding lies in [max(L, R) - STAGES, max(L, R)) and is its stage's last.
-template <int STAGES>
-__device__ __forceinline__ void drain_pair_stages(uint64_t* full, uint32_t stage_bytes, uint32_t L, uint32_t R) {
+template <int STAGES, class UseBytes>
+__device__ __forceinline__ void drain_pair_stages(uint64_t* full, UseBytes use_bytes, uint32_t L, uint32_t R) {
   const uint32_t hi = L > R ? L : R;
   for (uint32_t i = hi > (uint32_t)STAGES ? hi - STAGES : 0; i < hi; ++i) {
     const uint32_t s = i % STAGES, par = (i / STAGES) & 1;
     if (i >= L)
-      mbar_expect_tx(&full[s], stage_bytes);
+      mbar_expect_tx(&full[s], use_bytes(i));
     else if (i >= R)
-      mbar_complete_tx(&full[s], stage_bytes);
+      mbar_complete_tx(&full[s], use_bytes(i));
     mbar_wait_drain(&full[s], par);
   }
+}
+
+// One CTA's bytes in stage use i of this pair (a column slice loads a narrower B box).
+__device__ __forceinline__ uint32_t pair_use_bytes(const GemmArgs& a, int pair, int npairs, uint32_t i, int bn,
+                                                   uint32_t a_bytes, uint32_t b_bytes, int bk) {
+  for (int t = pair; t < a.total_items; t += npairs) {
+    int pi, m0, n0, width;
+    decode_item2(a, t, bn, pi, m0, n0, width);
+    const uint32_t kb = (uint32_t)(a.p[pi].K / bk);
+    if (i < kb) return a_bytes + (width == bn ? b_bytes : (uint32_t)(width / 2) * 128u);
+    i -= kb;
+  }
+  return a_bytes + b_bytes;
 }
 
 template <int BN, int EPI>
@@ -571,6 +607,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
     gemm2_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                     const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ CUtensorMap tmC1,
+                    const __grid_constant__ CUtensorMap tmB0n, const __grid_constant__ CUtensorMap tmB1n,
                     const __grid_constant__ GemmArgs args) {
   using C = Gemm2Cfg<BN, EPI>;
   constexpr int STAGES = C::STAGES;
@@ -612,6 +649,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
       tma_prefetch_desc(&tmA1);
       tma_prefetch_desc(&tmB1);
     }
+    if (args.tail_split > 1) {
+      tma_prefetch_desc(&tmB0n);
+      if (args.num_problems > 1) tma_prefetch_desc(&tmB1n);
+    }
   }
   if constexpr (EPI == EPI_QKV) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) {
@@ -635,20 +676,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
       bool ok = true;
-      for (int t = pair; t < args.total_tiles && ok; t += npairs) {
-        int pi, m0, n0;
-        decode_tile2(args, t, BN, pi, m0, n0);
+      for (int t = pair; t < args.total_items && ok; t += npairs) {
+        int pi, m0, n0, width;
+        decode_item2(args, t, BN, pi, m0, n0, width);
+        const bool slice = width < BN;
         const CUtensorMap* mA = pi ? &tmA1 : &tmA0;
-        const CUtensorMap* mB = pi ? &tmB1 : &tmB0;
+        const CUtensorMap* mB = slice ? (pi ? &tmB1n : &tmB0n) : (pi ? &tmB1 : &tmB0);
+        const uint32_t bytes = C::A_BYTES + (slice ? (uint32_t)(width / 2) * 128u : C::B_BYTES);
         const int kblocks = args.p[pi].K / C::BK;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, args.err)) {
             ok = false;
             break;
           }
-          if (rank == 0) mbar_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          if (rank == 0) mbar_expect_tx(&full[stage], 2 * bytes);
           tma_load_2d_pair(sA + stage * C::A_BYTES, mA, &full[stage], kb * C::BK, m0 + 128 * (int)rank);
-          tma_load_2d_pair(sB + stage * C::B_BYTES, mB, &full[stage], kb * C::BK, n0 + (BN / 2) * (int)rank);
+          // a column slice loads its own width / 2 rows through the narrow map
+          tma_load_2d_pair(sB + stage * C::B_BYTES, mB, &full[stage], kb * C::BK, n0 + (width / 2) * (int)rank);
           ++prod_issued;
           if (++stage == STAGES) {
             stage = 0;
@@ -663,13 +707,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16(256, BN);
       uint32_t stage = 0, phase = 0;
       int li = 0;
       bool ok = true;
-      for (int t = pair; t < args.total_tiles && ok; t += npairs, ++li) {
-        int pi, m0, n0;
-        decode_tile2(args, t, BN, pi, m0, n0);
+      for (int t = pair; t < args.total_items && ok; t += npairs, ++li) {
+        int pi, m0, n0, width;
+        decode_item2(args, t, BN, pi, m0, n0, width);
+        const uint32_t idesc = umma_idesc_bf16(256, width);
         const int kblocks = args.p[pi].K / C::BK;
         const uint32_t acc = li & 1;
         const uint32_t use = li >> 1;
@@ -709,19 +753,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
     uint32_t slot = 0;
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
     int li = 0;
-    for (int t = pair; t < args.total_tiles; t += npairs, ++li) {
-      int pi, m0, n0;
-      decode_tile2(args, t, BN, pi, m0, n0);
+    for (int t = pair; t < args.total_items; t += npairs, ++li) {
+      int pi, m0, n0, width;
+      decode_item2(args, t, BN, pi, m0, n0, width);
       const uint32_t acc = li & 1;
       const uint32_t use = li >> 1;
       const int row0 = m0 + 128 * (int)rank + quarter * 32;
       float4 pre[16];
-      epilogue_prefetch<BN, EPI>(args.p[pi], row0 + lane, n0, part, C::EPI_PARTS, pre);
+      epilogue_prefetch<BN, EPI>(args.p[pi], row0 + lane, n0, part, C::EPI_PARTS, pre, width);
       if (!mbar_wait(&tfull[acc], use & 1, args.err)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16) + acc * BN;
       epilogue_tile<BN, EPI, C::EPI_SLOTS>(args.p[pi], pi ? &tmC1 : &tmC0, row0 + lane, row0, n0, taddr, slots,
-                                           slot, sAux + pi * 128, pre, part, C::EPI_PARTS);
+                                           slot, sAux + pi * 128, pre, part, C::EPI_PARTS, width);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + acc * 8);
@@ -735,7 +779,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
   tc_fence_before();
   cluster_sync_all();          // every role of both CTAs has left its loop; rank 1's count is in place
   if (warp == 0 && lane == 0 && rank == 0 && (!prod_ok || err_raised(args.err)))
-    drain_pair_stages<STAGES>(full, C::STAGE_BYTES, prod_issued, *peer_issued);
+    drain_pair_stages<STAGES>(
+        full,
+        [&](uint32_t i) { return pair_use_bytes(args, pair, npairs, i, BN, C::A_BYTES, C::B_BYTES, C::BK); },
+        prod_issued, *peer_issued);
   cluster_sync_all();          // no MMA, TMA or remote arrive of the pair is still in flight
   if (warp == 1) {
     tc_fence_after();

@@ -43,6 +43,9 @@ struct StreamW {
   QW q_qkv, q_out, q_w13, q_w2;          // 4-bit weights (weight_bits = 4)
   float *b_qkv, *b_out, *b_w13, *b_w2, *gq, *gk;
   CUtensorMap t_qkv, t_out, t_w13, t_w2;
+  // the same weights with B boxes for 2- and 4-way column slices of a tile (the tail
+  // round of a CTA-pair launch; see launch_gemm_pair)
+  CUtensorMap n_qkv[2], n_out[2], n_w13[2], n_w2[2];
   // a bias that is absent or all zero is not added at all
   bool has_b_qkv = false, has_b_out = false, has_b_w13 = false, has_b_w2 = false;
 };
@@ -507,6 +510,15 @@ static lens_status make_weight_maps(lens_dit* h) {
            encode_tmap_bf16(&s.t_out, s.out, D, D, D, kBnOut / 2) &&
            encode_tmap_bf16(&s.t_w13, s.w13, 2 * kMlp, D, D, kBnW13 / 2) &&
            encode_tmap_bf16(&s.t_w2, s.w2, D, kMlp, kMlp, kBnW2 / 2);
+  for (auto& b : h->blk)
+    for (auto& s : b.s)
+      for (int i = 0; i < 2; ++i) {   // half of a 2- or 4-way column slice per CTA
+        const int q = 4 << i;
+        ok = ok && encode_tmap_bf16(&s.n_qkv[i], s.qkv, 3 * D, D, D, kBnQkv / q) &&
+             encode_tmap_bf16(&s.n_out[i], s.out, D, D, D, kBnOut / q) &&
+             encode_tmap_bf16(&s.n_w13[i], s.w13, 2 * kMlp, D, D, kBnW13 / q) &&
+             encode_tmap_bf16(&s.n_w2[i], s.w2, D, kMlp, kMlp, kBnW2 / q);
+      }
   return ok ? LENS_OK : LENS_ERR_CUDA;
 }
 
@@ -666,13 +678,15 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       p.eps = eps;
       a.p[s] = p;
     }
-    if (h->w4)
+    if (h->w4) {
       LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_w4(256, kBnQkvW4, EPI_QKV, false, &am.a_img, nullptr, &wi.q_qkv.tq, &wi.q_qkv.ts,
                             np > 1 ? &am.a_txt : nullptr, nullptr, np > 1 ? &wt.q_qkv.tq : nullptr, np > 1 ? &wt.q_qkv.ts : nullptr,
                             nullptr, nullptr, a, h->sms, st));
-    else
+    } else {
+      const NarrowB nb{{&wi.n_qkv[0], &wi.n_qkv[1]}, {&wt.n_qkv[0], &wt.n_qkv[1]}};
       LENS_LAUNCH(h, LENS_KERNEL_GEMM_QKV, st, launch_gemm_pair(kBnQkv, EPI_QKV, &am.a_img, &wi.t_qkv, np > 1 ? &am.a_txt : nullptr,
-                            np > 1 ? &wt.t_qkv : nullptr, nullptr, nullptr, a, h->sms, st));
+                            np > 1 ? &wt.t_qkv : nullptr, nullptr, nullptr, a, h->sms, st, &nb));
+    }
   }
   LENS_LAUNCH(h, LENS_KERNEL_ATTENTION, st, launch_joint_attention(h->q, h->k, h->v, B, kHeads, Nt, Ni, h->o_txt, h->o_img, tl, h->err, st));
   {
@@ -689,13 +703,15 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       p.rows_per_batch = s == 0 ? Ni : Nt;
       a.p[s] = p;
     }
-    if (h->w4)
+    if (h->w4) {
       LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm_w4(256, kBnResW4, EPI_RESID, false, &am.o_img, nullptr, &wi.q_out.tq, &wi.q_out.ts,
                             np > 1 ? &am.o_txt : nullptr, nullptr, np > 1 ? &wt.q_out.tq : nullptr, np > 1 ? &wt.q_out.ts : nullptr,
                             &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
-    else
+    } else {
+      const NarrowB nb{{&wi.n_out[0], &wi.n_out[1]}, {&wt.n_out[0], &wt.n_out[1]}};
       LENS_LAUNCH(h, LENS_KERNEL_GEMM_OUT, st, launch_gemm_pair(kBnOut, EPI_RESID, &am.o_img, &wi.t_out, np > 1 ? &am.o_txt : nullptr,
-                            np > 1 ? &wt.t_out : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
+                            np > 1 ? &wt.t_out : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st, &nb));
+    }
   }
   // MLP branch
   {
@@ -713,13 +729,15 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       p.bias = w.has_b_w13 ? w.b_w13 : nullptr;
       a.p[s] = p;
     }
-    if (h->w4)
+    if (h->w4) {
       LENS_LAUNCH(h, LENS_KERNEL_GEMM_W13, st, launch_gemm_w4(256, kBnW13W4, EPI_SWIGLU, false, &am.a_img, nullptr, &wi.q_w13.tq, &wi.q_w13.ts,
                             np > 1 ? &am.a_txt : nullptr, nullptr, np > 1 ? &wt.q_w13.tq : nullptr, np > 1 ? &wt.q_w13.ts : nullptr,
                             &am.uo_img, np > 1 ? &am.uo_txt : nullptr, a, h->sms, st));
-    else
+    } else {
+      const NarrowB nb{{&wi.n_w13[0], &wi.n_w13[1]}, {&wt.n_w13[0], &wt.n_w13[1]}};
       LENS_LAUNCH(h, LENS_KERNEL_GEMM_W13, st, launch_gemm_pair(kBnW13, EPI_SWIGLU, &am.a_img, &wi.t_w13, np > 1 ? &am.a_txt : nullptr,
-                            np > 1 ? &wt.t_w13 : nullptr, &am.uo_img, np > 1 ? &am.uo_txt : nullptr, a, h->sms, st));
+                            np > 1 ? &wt.t_w13 : nullptr, &am.uo_img, np > 1 ? &am.uo_txt : nullptr, a, h->sms, st, &nb));
+    }
   }
   {
     GemmArgs a = make_args(h->err);
@@ -735,13 +753,15 @@ static lens_status run_block(lens_dit* h, int i, float* hi, float* ht, int B, in
       p.rows_per_batch = s == 0 ? Ni : Nt;
       a.p[s] = p;
     }
-    if (h->w4)
+    if (h->w4) {
       LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm_w4(256, kBnResW4, EPI_RESID, false, &am.u_img, nullptr, &wi.q_w2.tq, &wi.q_w2.ts,
                             np > 1 ? &am.u_txt : nullptr, nullptr, np > 1 ? &wt.q_w2.tq : nullptr, np > 1 ? &wt.q_w2.ts : nullptr,
                             &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
-    else
+    } else {
+      const NarrowB nb{{&wi.n_w2[0], &wi.n_w2[1]}, {&wt.n_w2[0], &wt.n_w2[1]}};
       LENS_LAUNCH(h, LENS_KERNEL_GEMM_W2, st, launch_gemm_pair(kBnW2, EPI_RESID, &am.u_img, &wi.t_w2, np > 1 ? &am.u_txt : nullptr,
-                            np > 1 ? &wt.t_w2 : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st));
+                            np > 1 ? &wt.t_w2 : nullptr, &am.h_img, np > 1 ? &am.h_txt : nullptr, a, h->sms, st, &nb));
+    }
   }
   return LENS_OK;
 }
