@@ -191,13 +191,20 @@ class ClockSampler:
         self.uuid = uuid
         self.proc = None
         self.lines = []
+        self.first = 0
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # the query tool takes a while to start: begin the region once it samples, and
+            # keep only the samples from the region on
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 3.0:
+                time.sleep(0.005)
+            self.first = len(self.lines)
         except OSError:
             self.proc = None
         return self
@@ -208,6 +215,10 @@ class ClockSampler:
 
     def __exit__(self, *a):
         if self.proc:
+            # a region shorter than the sampling interval takes the first sample after it
+            t0 = time.time()
+            while len(self.lines) <= self.first and time.time() - t0 < 1.0:
+                time.sleep(0.005)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -216,7 +227,7 @@ class ClockSampler:
 
     def summary(self) -> dict:
         rows = []
-        for l in self.lines:
+        for l in self.lines[self.first:]:
             f = [x.strip() for x in l.split(",")]
             if len(f) < 9 or (self.uuid and self.uuid not in f[0]):
                 continue
