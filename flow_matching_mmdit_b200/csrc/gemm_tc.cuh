@@ -668,7 +668,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
   cluster_sync_all();          // both CTAs' barriers initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  grid_dependency_sync();      // set-up above touched only shared memory, TMEM and weights
+  // Programmatic dependent launch: only the producer and the epilogue warps touch memory
+  // that kernels ahead in the stream write (the A operand; outputs, gates, biases), so
+  // only they wait for those kernels; the producer first issues the weight (B) loads of
+  // its first stages, which depend on no kernel.
+  grid_launch_dependents();
 
   uint32_t prod_issued = 0;    // producer thread: stage loads issued
   bool prod_ok = true;
@@ -676,6 +680,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
       bool ok = true;
+      // the first item's first stages (each stage's first use: nothing to wait for) get
+      // their B tiles now, their A tiles once the kernels ahead have finished
+      int npre = 0;
+      if (pair < args.total_items) {
+        int pi, m0, n0, width;
+        decode_item2(args, pair, BN, pi, m0, n0, width);
+        const bool slice = width < BN;
+        const CUtensorMap* mB = slice ? (pi ? &tmB1n : &tmB0n) : (pi ? &tmB1 : &tmB0);
+        const uint32_t bytes = C::A_BYTES + (slice ? (uint32_t)(width / 2) * 128u : C::B_BYTES);
+        const int kblocks = args.p[pi].K / C::BK;
+        npre = kblocks < STAGES ? kblocks : STAGES;
+        for (int kb = 0; kb < npre; ++kb) {
+          if (rank == 0) mbar_expect_tx(&full[kb], 2 * bytes);
+          tma_load_2d_pair(sB + kb * C::B_BYTES, mB, &full[kb], kb * C::BK, n0 + (width / 2) * (int)rank);
+        }
+      }
+      grid_dependency_wait();
       for (int t = pair; t < args.total_items && ok; t += npairs) {
         int pi, m0, n0, width;
         decode_item2(args, t, BN, pi, m0, n0, width);
@@ -685,6 +706,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
         const uint32_t bytes = C::A_BYTES + (slice ? (uint32_t)(width / 2) * 128u : C::B_BYTES);
         const int kblocks = args.p[pi].K / C::BK;
         for (int kb = 0; kb < kblocks; ++kb) {
+          if (t == pair && kb < npre) {   // armed and B issued above
+            tma_load_2d_pair(sA + stage * C::A_BYTES, mA, &full[stage], kb * C::BK, m0 + 128 * (int)rank);
+            ++prod_issued;
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+            continue;
+          }
           if (!mbar_wait(&empty[stage], phase ^ 1, args.err)) {
             ok = false;
             break;
@@ -747,6 +777,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
     }
     __syncwarp();
   } else {
+    grid_dependency_wait();                       // gates, biases and outputs follow earlier kernels
     const int quarter = warp & 3;                 // TMEM lanes 32 quarter .. + 31
     const int part = (warp - 2) >> 2;             // which part of the tile's columns
     uint8_t* slots = sEpi + (warp - 2) * C::EPI_SLOTS * C::EPI_SLOT;
