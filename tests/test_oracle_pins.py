@@ -580,6 +580,28 @@ def test_final_layer_closed_form():
     assert abs(o.final_layer(W1, h, temb, 0.0)[0, 0, 0] - ((2.0 + _silu(2.0)) * 1.2 + 0.25)) < 1e-14
 
 
+def test_modulation_closed_form():
+    """AdaLN projection of a block stream ([blog] "Overview": shift, scale and gate for
+    the attention and for the MLP; [mlx] "自适应调制": img_mod / txt_mod): Linear of
+    SiLU(temb), split into six hidden-size chunks in the order (shift1, scale1, gate1,
+    shift2, scale2, gate2).  Zero weights return the bias chunks in that order; one unit
+    weight adds SiLU(temb_k) at one output column, not temb_k and not SiLU of the sum."""
+    D = 3
+    bias = np.arange(6 * D, dtype=np.float64) * 0.5 - 2.0
+    temb = np.array([[0.4, -1.5, 2.5]])
+    Wz = o.Weights({"blk.mod.weight": np.zeros((6 * D, D)), "blk.mod.bias": bias})
+    parts = o.modulation(Wz, "blk.mod", temb, 6)
+    assert len(parts) == 6
+    for i, p in enumerate(parts):
+        assert p.shape == (1, D) and np.array_equal(p[0], bias[i * D:(i + 1) * D])
+    w = np.zeros((6 * D, D))
+    w[2 * D + 1, 2] = 1.0                     # gate1, column 1 reads temb_2
+    W1 = o.Weights({"blk.mod.weight": w, "blk.mod.bias": bias})
+    g1 = o.modulation(W1, "blk.mod", temb, 6)[2][0]
+    assert abs(g1[1] - (bias[2 * D + 1] + _silu(2.5))) < 1e-14
+    assert np.array_equal(g1[[0, 2]], bias[[2 * D, 2 * D + 2]])
+
+
 def test_timestep_embedding_mlp_closed_form():
     """temb = linear_2(SiLU(linear_1(e))) ([mlx] time_text_embed.timestep_embedder).  At
     t = 0 the features are [1 ... 1, 0 ... 0] (cos 0, sin 0), so unit rows in linear_1
