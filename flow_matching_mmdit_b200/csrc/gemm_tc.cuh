@@ -441,14 +441,14 @@ __global__ void __launch_bounds__(192, 1)
         const int kblocks = args.p[pi].K / C::BK;
         const uint32_t acc = li & 1;
         const uint32_t use = li >> 1;
-        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) {
+        if (!mbar_wait_sleep(&tempty[acc], (use & 1) ^ 1, args.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, args.err)) {
+          if (!mbar_wait_sleep(&full[stage], phase, args.err)) {
             ok = false;
             break;
           }
@@ -747,14 +747,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Gemm2Cfg<BN, EPI>::T
         const int kblocks = args.p[pi].K / C::BK;
         const uint32_t acc = li & 1;
         const uint32_t use = li >> 1;
-        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) {
+        if (!mbar_wait_sleep(&tempty[acc], (use & 1) ^ 1, args.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, args.err)) {
+          if (!mbar_wait_sleep(&full[stage], phase, args.err)) {
             ok = false;
             break;
           }

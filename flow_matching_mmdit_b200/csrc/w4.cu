@@ -266,14 +266,14 @@ __global__ void __launch_bounds__(kW4Threads, 1)
         const int kblocks = args.p[pi].K / C::BK;
         const uint32_t acc = li & 1;
         const uint32_t use = li >> 1;
-        if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, args.err)) {
+        if (!mbar_wait_sleep(&tempty[acc], (use & 1) ^ 1, args.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * MH * BN;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&bfull[stage], phase, args.err)) {
+          if (!mbar_wait_sleep(&bfull[stage], phase, args.err)) {
             ok = false;
             break;
           }
