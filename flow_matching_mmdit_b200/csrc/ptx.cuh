@@ -82,9 +82,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
 }
 
 // The same for an MMA-issuing thread, whose waits sit between its MMA issues: the
-// poll carries a suspend-time hint, so the thread sleeps until the phase completes
-// (or 20 us pass) instead of re-polling (a plain poll loop there measured 2.6 % slower
-// over the block GEMMs).  The flag and the watchdog are checked every 16 polls.
+// poll carries a suspend-time hint, so the thread may be suspended (up to 20 us a
+// poll) while the phase is incomplete instead of re-polling at once (the plain poll
+// loop there measured 3 % slower over the block GEMMs).  The flag and the watchdog
+// are checked every 16 polls.
 __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
